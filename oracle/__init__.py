@@ -1,0 +1,162 @@
+"""fp64 CPU oracle of the mixture-of-experts FFN block.
+
+TEST INFRASTRUCTURE ONLY.  The parity reference for the CUDA path: only the
+tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may
+import this package.  It shares no code with the CUDA library, and the library
+never calls it.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, fp64, one loop per token over
+the selected experts); this module builds it with gcc and marshals numpy arrays.
+bf16 tensors are passed as their raw 16-bit patterns (numpy ``uint16``).
+
+Parity pins (what fixes this oracle other than itself) are in
+``tests/test_oracle_pins.py``.  Value-level parity against the pages is
+unpinned: the pages print no worked numerical example for the block, so the
+values are pinned by closed forms, special cases and invariants only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+SOFTMAX, SIGMOID, SQRT_SOFTPLUS = 0, 1, 2
+SCORE_FNS = {"softmax": SOFTMAX, "sigmoid": SIGMOID, "sqrt_softplus": SQRT_SOFTPLUS}
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into liboracle.so (gcc, -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            i = ctypes.c_int
+            lib.oracle_moe_forward.restype = i
+            lib.oracle_moe_forward.argtypes = (
+                [i] * 7 + [P] * 3 + [P] * 6 + [i, i, ctypes.c_double] + [P, i, P, i] + [P] * 6 + [i])
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else ctypes.c_void_p(a.ctypes.data)
+
+
+def _u16(a, shape, name):
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"{name}: expected raw bf16 bits as uint16, got {a.dtype}")
+    if tuple(a.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(a.shape)}")
+    return a
+
+
+def forward(x, W_router, W_gate=None, W_up=None, W_down=None,
+            W_shared_gate=None, W_shared_up=None, W_shared_down=None,
+            expert_bias=None, *, k, score_fn="softmax", norm_topk=True, route_scale=1.0,
+            tokens=None, forced_idx=None, route_only=False, want_logits=False,
+            n_threads=None):
+    """Run the oracle.
+
+    Shapes (bf16 bit patterns as uint16): x [T,d], W_router [E,d],
+    W_gate/W_up [E,f,d], W_down [E,d,f], W_shared_gate/up [S,fs,d],
+    W_shared_down [S,d,fs]; expert_bias fp32 [E] or None.
+
+    ``tokens`` restricts evaluation to those token ids (outputs are in that
+    order); ``forced_idx`` [n,k] replaces the router's choice of experts (the
+    weights are then the scores of the forced experts, renormalised the same
+    way).  Returns a dict of float64/int32 numpy arrays: ``out`` [n,d],
+    ``topk_idx`` [n,k], ``topk_w`` [n,k], ``sel_keys`` [n,k+1] (selection keys
+    of the first k+1 experts in selection order), and with ``want_logits``
+    also ``logits`` and ``scores`` [n,E].
+    """
+    lib = _load()
+    T, d = x.shape
+    E = W_router.shape[0]
+    x = _u16(x, (T, d), "x")
+    W_router = _u16(W_router, (E, d), "W_router")
+    if route_only:
+        f, S, fs = 1, 0, 1
+    else:
+        f = W_gate.shape[1]
+        W_gate = _u16(W_gate, (E, f, d), "W_gate")
+        W_up = _u16(W_up, (E, f, d), "W_up")
+        W_down = _u16(W_down, (E, d, f), "W_down")
+        S = 0 if W_shared_gate is None else W_shared_gate.shape[0]
+        fs = 1 if S == 0 else W_shared_gate.shape[1]
+        if S:
+            W_shared_gate = _u16(W_shared_gate, (S, fs, d), "W_shared_gate")
+            W_shared_up = _u16(W_shared_up, (S, fs, d), "W_shared_up")
+            W_shared_down = _u16(W_shared_down, (S, d, fs), "W_shared_down")
+    if expert_bias is not None:
+        expert_bias = np.ascontiguousarray(expert_bias, dtype=np.float32)
+        if expert_bias.shape != (E,):
+            raise ValueError("expert_bias must be fp32 [E]")
+    if tokens is None:
+        tok = None
+        n = T
+    else:
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = int(tok.shape[0])
+    forced = None if forced_idx is None else np.ascontiguousarray(forced_idx, dtype=np.int32)
+    if forced is not None and forced.shape != (n, k):
+        raise ValueError("forced_idx must be [n_tokens, k]")
+
+    out = None if route_only else np.zeros((n, d), np.float64)
+    topk_idx = np.zeros((n, k), np.int32)
+    topk_w = np.zeros((n, k), np.float64)
+    sel_keys = np.zeros((n, k + 1), np.float64)
+    logits = np.zeros((n, E), np.float64) if want_logits else None
+    scores = np.zeros((n, E), np.float64) if want_logits else None
+    if n_threads is None:
+        n_threads = os.cpu_count() or 1
+    st = lib.oracle_moe_forward(
+        T, d, E, k, f, S, fs,
+        _ptr(x), _ptr(W_router), _ptr(expert_bias),
+        _ptr(W_gate), _ptr(W_up), _ptr(W_down),
+        _ptr(W_shared_gate), _ptr(W_shared_up), _ptr(W_shared_down),
+        SCORE_FNS[score_fn] if isinstance(score_fn, str) else int(score_fn),
+        int(bool(norm_topk)), float(route_scale),
+        _ptr(tok), n, _ptr(forced), int(bool(route_only)),
+        _ptr(out), _ptr(topk_idx), _ptr(topk_w), _ptr(sel_keys),
+        _ptr(logits), _ptr(scores), int(n_threads))
+    if st != 0:
+        raise ValueError(f"oracle_moe_forward failed with status {st}")
+    res = {"out": out, "topk_idx": topk_idx, "topk_w": topk_w, "sel_keys": sel_keys}
+    if want_logits:
+        res["logits"] = logits
+        res["scores"] = scores
+    return res
+
+
+def rel_gap(a, b):
+    """|a-b| / max(|a|,|b|), elementwise, 0 where both are 0."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    m = np.maximum(np.abs(a), np.abs(b))
+    with np.errstate(invalid="ignore", divide="ignore"):
+        g = np.where(m > 0, np.abs(a - b) / np.where(m > 0, m, 1.0), 0.0)
+    return g

@@ -1,0 +1,362 @@
+"""Pins of the fp64 oracle to things other than itself (CPU only).
+
+Each test checks the oracle against something the pages or the mathematics fix:
+hand-derived closed forms, brute force on tiny inputs, library routines that a
+special case reduces to (numpy matmul, scipy expit / logaddexp), identities and
+invariants.  Together they are chosen so that a dropped term, a wrong sign or
+index, or a transposed operand anywhere in the oracle fails at least one.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import expit
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bits(a):
+    """float array -> bf16 bits; only used on values that are exact in bf16 or
+    that the test then reads back through `widen`."""
+    from mixture_experts_ffn_16_b200.inputs import bf16_round
+    return bf16_round(np.asarray(a, np.float32))
+
+
+def widen(b):
+    """bf16 bits -> float64 (independent of the oracle's own widening)."""
+    return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def rand_case(rng, T, d, E, f, S=0, fs=64, w_std=0.3, x_std=1.0):
+    c = dict(x=bits(rng.normal(0, x_std, (T, d))),
+             W_router=bits(rng.normal(0, w_std, (E, d))),
+             W_gate=bits(rng.normal(0, w_std, (E, f, d))),
+             W_up=bits(rng.normal(0, w_std, (E, f, d))),
+             W_down=bits(rng.normal(0, w_std, (E, d, f))))
+    if S:
+        c.update(W_shared_gate=bits(rng.normal(0, w_std, (S, fs, d))),
+                 W_shared_up=bits(rng.normal(0, w_std, (S, fs, d))),
+                 W_shared_down=bits(rng.normal(0, w_std, (S, d, fs))))
+    return c
+
+
+def swiglu_dense(x, G, U, D):
+    """Textbook matrix form D (SiLU(G x) * (U x)) for x [T,d] (rows), numpy fp64."""
+    g = x @ G.T
+    u = x @ U.T
+    return (g * expit(g) * u) @ D.T
+
+
+# ---------------------------------------------------------------- golden cases
+
+def _eval(expr):
+    env = {"sigma": lambda z: 1.0 / (1.0 + math.exp(-z)),
+           "silu": lambda z: z / (1.0 + math.exp(-z)),
+           "exp": math.exp, "log": math.log, "sqrt": math.sqrt}
+    return float(eval(expr, {"__builtins__": {}}, env))
+
+
+def _load_cases():
+    with open(os.path.join(GOLDEN, "hand_cases.json")) as fh:
+        return json.load(fh)["cases"]
+
+
+@pytest.mark.parametrize("case", _load_cases(), ids=lambda c: c["name"])
+def test_hand_derived_cases(oracle_mod, case):
+    arr = {k: bits(np.array(case[k], np.float64)) for k in
+           ["x", "W_router", "W_gate", "W_up", "W_down"]}
+    for k in ["W_shared_gate", "W_shared_up", "W_shared_down"]:
+        arr[k] = bits(np.array(case[k], np.float64)) if k in case else None
+    # every input of a hand case must be exact in bf16
+    for k, v in arr.items():
+        if v is not None:
+            assert np.array_equal(widen(v), np.array(case[k], np.float64)), k
+    bias = np.array(case["expert_bias"], np.float32) if "expert_bias" in case else None
+    r = oracle_mod.forward(**arr, expert_bias=bias, k=case["k"], score_fn=case["score_fn"],
+                           norm_topk=case["norm_topk"], route_scale=case["route_scale"])
+    assert r["topk_idx"].tolist() == case["expected_idx"]
+    np.testing.assert_allclose(r["topk_w"][0], [_eval(e) for e in case["expected_w"]],
+                               rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(r["out"], [[_eval(e) for e in row] for row in case["expected_out"]],
+                               rtol=1e-13, atol=1e-14)
+
+
+def test_page_sizes_pin_decode_layer_volume():
+    """The Qwen3.5 MoE sizes printed on the pages: 60 layers x 512 experts x
+    3 matrices x 4096 x 1024 = 386.5B routed parameters, which fits inside the
+    397B total, and one such layer holds 12.88 GB of bf16 expert weights: the
+    volume the decode-shaped workload streams when every expert is touched."""
+    with open(os.path.join(GOLDEN, "page_sizes.json")) as fh:
+        v = {k: x["value"] for k, x in json.load(fh)["values"].items()}
+    routed = v["n_layers"] * v["n_experts"] * 3 * v["d_model"] * v["d_ff"]
+    assert abs(routed - 386.5e9) < 0.1e9 and routed < v["total_params"]
+    layer_bytes = v["n_experts"] * 3 * v["d_model"] * v["d_ff"] * 2
+    assert abs(layer_bytes - 12.88e9) < 0.01e9
+    assert abs(v["top_k"] / v["n_experts"] - v["active_fraction_text"]) < 0.001
+    from mixture_experts_ffn_16_b200.inputs import CONFIGS
+    c = CONFIGS["decode_sqrt_softplus"]
+    assert (c.E, c.f, c.d, c.k) == (v["n_experts"], v["d_ff"], v["d_model"], v["top_k"])
+
+
+# ---------------------------------------------------------------- router pins
+
+def test_logits_match_numpy_matmul(oracle_mod):
+    rng = np.random.default_rng(1)
+    c = rand_case(rng, 7, 40, 11, 8)
+    r = oracle_mod.forward(c["x"], c["W_router"], k=3, route_only=True, want_logits=True)
+    np.testing.assert_allclose(r["logits"], widen(c["x"]) @ widen(c["W_router"]).T,
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_score_closed_forms(oracle_mod):
+    """sigmoid(0)=1/2, sqrt(softplus(0))=sqrt(ln 2), equal logits -> softmax 1/E,
+    and library routines elsewhere (scipy expit, numpy logaddexp)."""
+    E, d = 6, 8
+    x = np.zeros((1, d), np.float64)
+    x[0, 0] = 1.0
+    Wr = np.zeros((E, d))
+    vals = np.array([0.0, 1.0, -2.0, 30.0, -30.0, 0.5])
+    Wr[:, 0] = vals
+    xb, Wb = bits(x), bits(Wr)
+    s_sig = oracle_mod.forward(xb, Wb, k=1, score_fn="sigmoid", route_only=True,
+                               want_logits=True)["scores"][0]
+    s_sp = oracle_mod.forward(xb, Wb, k=1, score_fn="sqrt_softplus", route_only=True,
+                              want_logits=True)["scores"][0]
+    assert s_sig[0] == 0.5
+    assert abs(s_sp[0] - math.sqrt(math.log(2.0))) < 1e-15
+    np.testing.assert_allclose(s_sig, expit(vals), rtol=1e-14)
+    np.testing.assert_allclose(s_sp, np.sqrt(np.logaddexp(0.0, vals)), rtol=1e-14)
+    s_sm = oracle_mod.forward(bits(np.zeros((1, d))), Wb, k=1, score_fn="softmax",
+                              route_only=True, want_logits=True)["scores"][0]
+    np.testing.assert_allclose(s_sm, np.full(E, 1.0 / E), rtol=1e-15)
+
+
+CASES = [(E, k) for E in (1, 2, 3, 5, 8, 16) for k in sorted({1, 2, E // 2 or 1, E}) if k <= E]
+
+
+@pytest.mark.parametrize("E,k", CASES)
+@pytest.mark.parametrize("score_fn", ["softmax", "sigmoid", "sqrt_softplus"])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_topk_brute_force(oracle_mod, E, k, score_fn, with_bias):
+    """Selection = full Python sort by (key desc, index asc) of the oracle's own
+    scores (+ bias for sigmoid / sqrt-softplus); ties are provoked by rounding
+    the router to a coarse grid."""
+    rng = np.random.default_rng(E * 100 + k * 7 + (3 if with_bias else 0))
+    T, d = 24, 6
+    x = bits(np.round(rng.normal(0, 1, (T, d)) * 2) / 2)
+    Wr = bits(np.round(rng.normal(0, 1, (E, d)) * 2) / 4)
+    bias = np.round(rng.normal(0, 0.5, E) * 4).astype(np.float32) / 4 if with_bias else None
+    r = oracle_mod.forward(x, Wr, expert_bias=bias, k=k, score_fn=score_fn, route_only=True,
+                           want_logits=True)
+    for t in range(T):
+        s = r["scores"][t]
+        key = s + (bias.astype(np.float64) if (bias is not None and score_fn != "softmax") else 0.0)
+        order = sorted(range(E), key=lambda e: (-key[e], e))
+        assert r["topk_idx"][t].tolist() == order[:k]
+        np.testing.assert_array_equal(r["sel_keys"][t][:min(k + 1, E)],
+                                      [key[e] for e in order[:k + 1]])
+
+
+def test_all_zero_router_ties_to_lowest_indices(oracle_mod):
+    x = bits(np.ones((3, 16)))
+    Wr = bits(np.zeros((9, 16)))
+    for fn in ["softmax", "sigmoid", "sqrt_softplus"]:
+        r = oracle_mod.forward(x, Wr, k=4, score_fn=fn, route_only=True)
+        assert r["topk_idx"].tolist() == [[0, 1, 2, 3]] * 3
+        np.testing.assert_allclose(r["topk_w"], 0.25, rtol=1e-15)
+
+
+@pytest.mark.parametrize("score_fn", ["softmax", "sigmoid", "sqrt_softplus"])
+@pytest.mark.parametrize("scale", [1.0, 2.5])
+def test_renormalised_weights_sum_to_route_scale(oracle_mod, score_fn, scale):
+    rng = np.random.default_rng(5)
+    c = rand_case(rng, 20, 32, 12, 8)
+    bias = rng.normal(0, 0.1, 12).astype(np.float32)
+    r = oracle_mod.forward(c["x"], c["W_router"], expert_bias=bias, k=5, score_fn=score_fn,
+                           norm_topk=True, route_scale=scale, route_only=True)
+    np.testing.assert_allclose(r["topk_w"].sum(1), scale, rtol=1e-14)
+
+
+def test_softmax_renorm_equals_softmax_over_selected_logits(oracle_mod):
+    """softmax-then-renormalise over the k picks == softmax of the k picked
+    logits alone (the full denominator cancels)."""
+    rng = np.random.default_rng(6)
+    c = rand_case(rng, 30, 24, 16, 8)
+    r = oracle_mod.forward(c["x"], c["W_router"], k=4, score_fn="softmax", route_only=True)
+    L = widen(c["x"]) @ widen(c["W_router"]).T
+    for t in range(30):
+        l_sel = L[t, r["topk_idx"][t]]
+        ref = np.exp(l_sel - l_sel.max())
+        np.testing.assert_allclose(r["topk_w"][t], ref / ref.sum(), rtol=1e-12)
+
+
+def test_unnormalised_weights_are_raw_scores(oracle_mod):
+    rng = np.random.default_rng(7)
+    c = rand_case(rng, 10, 24, 16, 8)
+    L = widen(c["x"]) @ widen(c["W_router"]).T
+    r = oracle_mod.forward(c["x"], c["W_router"], k=3, score_fn="sigmoid", norm_topk=False,
+                           route_only=True)
+    np.testing.assert_allclose(r["topk_w"], expit(np.take_along_axis(L, r["topk_idx"], 1)),
+                               rtol=1e-12)
+    r = oracle_mod.forward(c["x"], c["W_router"], k=3, score_fn="softmax", norm_topk=False,
+                           route_only=True)
+    P = np.exp(L - L.max(1, keepdims=True))
+    P /= P.sum(1, keepdims=True)
+    np.testing.assert_allclose(r["topk_w"], np.take_along_axis(P, r["topk_idx"], 1), rtol=1e-12)
+
+
+@pytest.mark.parametrize("score_fn", ["sigmoid", "sqrt_softplus"])
+def test_bias_changes_selection_never_weights(oracle_mod, score_fn):
+    rng = np.random.default_rng(8)
+    E, k = 16, 4
+    c = rand_case(rng, 25, 32, E, 8)
+    base = oracle_mod.forward(c["x"], c["W_router"], k=k, score_fn=score_fn, route_only=True,
+                              want_logits=True)
+    # (a) a bias that keeps every token's selection keeps the weights bit-identical
+    tiny = np.full(E, 1e-300, np.float32)  # rounds to 0 in fp32: leaves keys unchanged
+    same = oracle_mod.forward(c["x"], c["W_router"], expert_bias=tiny, k=k, score_fn=score_fn,
+                              route_only=True)
+    assert np.array_equal(same["topk_idx"], base["topk_idx"])
+    assert np.array_equal(same["topk_w"], base["topk_w"])
+    # (b) a huge bias on one expert forces it first; its weight stays s_e / sum of picked s
+    forced_e = 11
+    big = np.zeros(E, np.float32)
+    big[forced_e] = 1e6
+    r = oracle_mod.forward(c["x"], c["W_router"], expert_bias=big, k=k, score_fn=score_fn,
+                           route_only=True)
+    assert (r["topk_idx"][:, 0] == forced_e).all()
+    s = base["scores"]
+    picked = np.take_along_axis(s, r["topk_idx"], 1)
+    np.testing.assert_allclose(r["topk_w"], picked / picked.sum(1, keepdims=True), rtol=1e-14)
+    # (c) biases that reorder the picks re-derive weights from the unbiased scores only
+    b = rng.normal(0, 0.3, E).astype(np.float32)
+    r = oracle_mod.forward(c["x"], c["W_router"], expert_bias=b, k=k, score_fn=score_fn,
+                           route_only=True)
+    picked = np.take_along_axis(s, r["topk_idx"], 1)
+    np.testing.assert_allclose(r["topk_w"], picked / picked.sum(1, keepdims=True), rtol=1e-14)
+    assert not np.array_equal(r["topk_idx"], base["topk_idx"])
+
+
+def test_softmax_ignores_bias(oracle_mod):
+    rng = np.random.default_rng(9)
+    c = rand_case(rng, 10, 16, 8, 8)
+    b = rng.normal(0, 5, 8).astype(np.float32)
+    a = oracle_mod.forward(c["x"], c["W_router"], k=2, score_fn="softmax", route_only=True)
+    z = oracle_mod.forward(c["x"], c["W_router"], expert_bias=b, k=2, score_fn="softmax",
+                           route_only=True)
+    assert np.array_equal(a["topk_idx"], z["topk_idx"]) and np.array_equal(a["topk_w"], z["topk_w"])
+
+
+# ---------------------------------------------------------------- expert pins
+
+@pytest.mark.parametrize("S", [0, 1])
+def test_single_expert_is_dense_swiglu(oracle_mod, S):
+    """E=1, k=1, softmax: w=1, so the block is a dense SwiGLU FFN (+ shared),
+    checked against the numpy matrix form with d != f != fs to catch transposes."""
+    rng = np.random.default_rng(10 + S)
+    c = rand_case(rng, 9, 48, 1, 80, S=S, fs=24)
+    r = oracle_mod.forward(**c, k=1)
+    ref = swiglu_dense(widen(c["x"]), widen(c["W_gate"][0]), widen(c["W_up"][0]),
+                       widen(c["W_down"][0]))
+    if S:
+        ref += swiglu_dense(widen(c["x"]), widen(c["W_shared_gate"][0]),
+                            widen(c["W_shared_up"][0]), widen(c["W_shared_down"][0]))
+    assert (r["topk_idx"] == 0).all() and (r["topk_w"] == 1.0).all()
+    np.testing.assert_allclose(r["out"], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_out_is_weighted_sum_of_dense_experts(oracle_mod):
+    """out[t] = sum_j w_j SwiGLU_{e_j}(x_t) + shared, with each expert's output
+    from the numpy matrix form: pins the combine (every term, its weight, its sign)."""
+    rng = np.random.default_rng(12)
+    E, k, S = 6, 3, 2
+    c = rand_case(rng, 11, 32, E, 40, S=S, fs=16)
+    bias = rng.normal(0, 0.2, E).astype(np.float32)
+    r = oracle_mod.forward(**c, expert_bias=bias, k=k, score_fn="sqrt_softplus", route_scale=2.5)
+    X = widen(c["x"])
+    Y = [swiglu_dense(X, widen(c["W_gate"][e]), widen(c["W_up"][e]), widen(c["W_down"][e]))
+         for e in range(E)]
+    Ysh = sum(swiglu_dense(X, widen(c["W_shared_gate"][s]), widen(c["W_shared_up"][s]),
+                           widen(c["W_shared_down"][s])) for s in range(S))
+    ref = Ysh.copy()
+    for t in range(11):
+        for j in range(k):
+            ref[t] += r["topk_w"][t, j] * Y[r["topk_idx"][t, j]][t]
+    np.testing.assert_allclose(r["out"], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_two_shared_experts_equal_one_concatenated(oracle_mod):
+    """S=2 shared experts of width fs == one shared expert of width 2*fs whose
+    gate/up rows and down columns are the two stacked."""
+    rng = np.random.default_rng(13)
+    c = rand_case(rng, 8, 32, 4, 16, S=2, fs=24)
+    r2 = oracle_mod.forward(**c, k=2)
+    c1 = dict(c)
+    c1["W_shared_gate"] = np.concatenate([c["W_shared_gate"][0], c["W_shared_gate"][1]], 0)[None]
+    c1["W_shared_up"] = np.concatenate([c["W_shared_up"][0], c["W_shared_up"][1]], 0)[None]
+    c1["W_shared_down"] = np.concatenate([c["W_shared_down"][0], c["W_shared_down"][1]], 1)[None]
+    r1 = oracle_mod.forward(**c1, k=2)
+    np.testing.assert_allclose(r1["out"], r2["out"], rtol=1e-12, atol=1e-13)
+
+
+def test_token_permutation_equivariance(oracle_mod):
+    rng = np.random.default_rng(14)
+    c = rand_case(rng, 17, 32, 8, 16, S=1, fs=16)
+    r = oracle_mod.forward(**c, k=3, score_fn="sigmoid")
+    p = rng.permutation(17)
+    cp = dict(c)
+    cp["x"] = c["x"][p]
+    rp = oracle_mod.forward(**cp, k=3, score_fn="sigmoid")
+    assert np.array_equal(rp["topk_idx"], r["topk_idx"][p])
+    assert np.array_equal(rp["out"], r["out"][p])
+    # the token subset path evaluates the same tokens identically
+    sub = oracle_mod.forward(**c, k=3, score_fn="sigmoid", tokens=p[:5])
+    assert np.array_equal(sub["out"], r["out"][p[:5]])
+
+
+def test_doubling_w_down_doubles_out_exactly(oracle_mod):
+    rng = np.random.default_rng(15)
+    c = rand_case(rng, 6, 32, 5, 16, S=1, fs=16)
+    r = oracle_mod.forward(**c, k=2)
+    c2 = dict(c)
+    c2["W_down"] = bits(2 * widen(c["W_down"]))
+    c2["W_shared_down"] = bits(2 * widen(c["W_shared_down"]))
+    r2 = oracle_mod.forward(**c2, k=2)
+    assert np.array_equal(r2["out"], 2 * r["out"])
+    assert np.array_equal(r2["topk_idx"], r["topk_idx"])
+
+
+def test_forced_indices_reproduce_own_choice(oracle_mod):
+    rng = np.random.default_rng(16)
+    c = rand_case(rng, 10, 32, 7, 16, S=1, fs=16)
+    r = oracle_mod.forward(**c, k=3)
+    f = oracle_mod.forward(**c, k=3, forced_idx=r["topk_idx"])
+    assert np.array_equal(f["out"], r["out"]) and np.array_equal(f["topk_w"], r["topk_w"])
+    # forcing a different set changes the output by exactly the swapped terms
+    forced = r["topk_idx"].copy()
+    forced[:, 2] = (forced[:, 2] + 1) % 7
+    forced[:, 2] = np.where(np.isin(forced[:, 2], forced[:, :2]), (forced[:, 2] + 3) % 7,
+                            forced[:, 2])
+    g = oracle_mod.forward(**c, k=3, forced_idx=forced)
+    assert np.array_equal(g["topk_idx"], forced)
+
+
+def test_threads_do_not_change_results(oracle_mod):
+    rng = np.random.default_rng(17)
+    c = rand_case(rng, 33, 32, 9, 16, S=1, fs=16)
+    a = oracle_mod.forward(**c, k=4, n_threads=1)
+    b = oracle_mod.forward(**c, k=4, n_threads=5)
+    for key in ("out", "topk_idx", "topk_w", "sel_keys"):
+        assert np.array_equal(a[key], b[key])
+
+
+def test_invalid_arguments_rejected(oracle_mod):
+    rng = np.random.default_rng(18)
+    c = rand_case(rng, 4, 16, 3, 8)
+    with pytest.raises(ValueError):
+        oracle_mod.forward(**c, k=4)           # k > E
+    with pytest.raises(ValueError):
+        oracle_mod.forward(**c, k=1, tokens=[0, 9])   # token out of range
