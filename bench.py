@@ -1,0 +1,364 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE FFN block on B200: one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is one pass of the whole block (router GEMM, top-k, permute, gate/up
+GEMM, down GEMM, combine) over one batch of T tokens whose inputs are already
+in HBM.  Default workload: prefill with a softmax top-8 router (T=4096,
+d=2048, E=256, d_ff=512, one shared expert of 512), seeded synthetic inputs.
+With N GPUs (torchrun) every rank runs its own replica on its own batch
+(weak scaling, no collective on the data path); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the slow plain definition) on a
+bounded sample of the same workload on rank 0; other ranks exit at once.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from mixture_experts_ffn_16_b200 import api  # noqa: E402
+from mixture_experts_ffn_16_b200.inputs import CONFIGS, make_inputs, oracle_args  # noqa: E402
+from mixture_experts_ffn_16_b200.roofline import block_cost, kernel_costs, measured_peaks  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec at 1 B200; % bf16 tensor peak (prefill) / % HBM BW (decode)"
+STAGES = ["route", "permute", "gate_up", "down", "combine"]
+LAUNCHES_PER_STEP = {"route": 2, "permute": 3, "gate_up": 1, "down": 1, "combine": 1}
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="prefill_softmax", choices=list(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, device_index, period_s=0.01):
+        self.samples = []
+        self.max_mhz = None
+        self.period = period_s
+        self.dev = device_index
+        self._stop = threading.Event()
+        self._t = None
+        self.error = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            get_r = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def run():
+                while True:
+                    try:
+                        self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                             int(get_r(h))))
+                    except Exception as e:  # noqa: BLE001
+                        self.error = str(e)
+                    if self._stop.wait(self.period):
+                        break
+            self._t = threading.Thread(target=run, daemon=True)
+            self._t.start()
+        except Exception as e:  # noqa: BLE001
+            self.error = str(e)
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "error": self.error}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[1]
+        reasons = [name for b, name in REASON_BITS.items() if bits & b]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_oracle_rate(cfg, host, target_s, seed=12345):
+    """Time the oracle on a seeded token sample sized to about target_s seconds."""
+    import oracle
+    oracle.build()
+    threads = os.cpu_count() or 1
+    rng = np.random.default_rng(seed)
+    n = min(cfg.T, max(threads, 8))
+    t0 = time.perf_counter()
+    oracle.forward(**host, k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk,
+                   route_scale=cfg.route_scale, tokens=rng.choice(cfg.T, n, replace=False).astype(np.int32),
+                   n_threads=threads)
+    dt = time.perf_counter() - t0
+    n2 = int(min(cfg.T, max(n, n * target_s / max(dt, 1e-6))))
+    toks = rng.choice(cfg.T, n2, replace=False).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.forward(**host, k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk,
+                   route_scale=cfg.route_scale, tokens=toks, n_threads=threads)
+    dt = time.perf_counter() - t0
+    return n2 / dt, threads, n2, dt
+
+
+def run_reference(args, cfg):
+    """fp64 oracle on the host cores, per step a bounded token sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(cfg, device=dev)
+    host = oracle_args(inp)
+    del inp
+    threads = os.cpu_count() or 1
+    rng = np.random.default_rng(777)
+    # calibrate, then size each step so that warmup + steps take about 120 s
+    n0 = min(cfg.T, max(threads, 4))
+    t0 = time.perf_counter()
+    oracle.forward(**host, k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk,
+                   route_scale=cfg.route_scale, tokens=rng.choice(cfg.T, n0, replace=False).astype(np.int32),
+                   n_threads=threads)
+    rate = n0 / (time.perf_counter() - t0)
+    per_step_s = 120.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(cfg.T, rate * per_step_s)))
+    total_tok, total_s = 0, 0.0
+    for i in range(args.warmup + args.steps):
+        toks = rng.choice(cfg.T, n, replace=False).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.forward(**host, k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk,
+                       route_scale=cfg.route_scale, tokens=toks, n_threads=threads)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            total_tok += n
+            total_s += dt
+    value = total_tok / total_s
+    sample = f"{n} seeded tokens of {cfg.name} per step (full block per token, fp64)"
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "E": cfg.E, "k": cfg.k,
+                       "d_ff": cfg.f, "n_shared": cfg.S, "d_ff_shared": cfg.fs, "score_fn": cfg.score_fn},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, cfg):
+    world, rank, local = dist_setup(args.gpus)
+    api.load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    inp = make_inputs(cfg, device=dev, seed=cfg.seed + 1000 * rank)
+    layer = api.MoELayer(cfg, inp, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    s = layer.shape
+
+    def step(ev=None):
+        t, c = inp, cfg
+        if ev is not None:
+            ev[0].record(stream)
+        api.moe_route(s, t["x"], t["W_router"], t["expert_bias"], c.score_fn, c.norm_topk, c.route_scale,
+                      layer.topk_idx, layer.topk_w, layer.workspace, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        api.moe_permute(s, layer.topk_idx, layer.topk_w, layer.workspace, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        api.moe_expert_gate_up(s, t["x"], t["W_gate"], t["W_up"], t["W_shared_gate"], t["W_shared_up"],
+                               layer.workspace, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        api.moe_expert_down(s, t["W_down"], t["W_shared_down"], layer.workspace, stream)
+        if ev is not None:
+            ev[4].record(stream)
+        api.moe_combine(s, layer.out, layer.workspace, stream)
+        if ev is not None:
+            ev[5].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    st = api.moe_device_status(layer.workspace, stream)
+    if st != api.MOE_OK:
+        raise RuntimeError(f"device status after warm-up: {api.status_string(st)}")
+    idx_host = layer.topk_idx.cpu().numpy()
+    touched = int((np.bincount(idx_host.ravel(), minlength=cfg.E) > 0).sum())
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        for i in range(K):
+            step(evs[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = evs[0][0].elapsed_time(evs[-1][5])
+    stage_ms = {name: 0.0 for name in STAGES}
+    for ev in evs:
+        for j, name in enumerate(STAGES):
+            stage_ms[name] += ev[j].elapsed_time(ev[j + 1])
+    stage_avg_us = {n: 1e3 * v / K for n, v in stage_ms.items()}
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    st = api.moe_device_status(layer.workspace, stream)
+    if st != api.MOE_OK:
+        raise RuntimeError(f"device status after timing: {api.status_string(st)}")
+
+    # end to end through the public host-buffer entry point
+    e2e = None
+    if not args.no_e2e:
+        xh = inp["x"].cpu().pin_memory()
+        oh = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16).pin_memory()
+        ih = torch.empty((cfg.T, cfg.k), dtype=torch.int32).pin_memory()
+        wh = torch.empty((cfg.T, cfg.k), dtype=torch.float32).pin_memory()
+
+        def host_step():
+            api.moe_forward_host(s, xh, inp["W_router"], inp["expert_bias"], inp["W_gate"], inp["W_up"],
+                                 inp["W_down"], inp["W_shared_gate"], inp["W_shared_up"], inp["W_shared_down"],
+                                 cfg.score_fn, cfg.norm_topk, cfg.route_scale, oh, ih, wh, layer.workspace, stream)
+        for _ in range(max(3, args.warmup)):
+            host_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(K):
+            host_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": world * cfg.T * K / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": cfg.T * cfg.d * 2,
+               "d2h_bytes_per_step": cfg.T * cfg.d * 2 + cfg.T * cfg.k * 8}
+
+    value = world * cfg.T * K / (elapsed_ms / 1e3)
+    peaks = measured_peaks()
+    costs = kernel_costs(cfg, touched)
+    dom = max(STAGES, key=lambda n: stage_avg_us[n])
+    fl, by = costs[dom]
+    t_s = stage_avg_us[dom] * 1e-6
+    t_mem = by / (peaks["hbm_gbs"] * 1e9)
+    t_math = fl / (peaks["bf16_tflops"] * 1e12)
+    if t_math > t_mem:
+        roof = {"bound": "tensor", "achieved": fl / t_s / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": by / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["algorithmic_bytes"] = by
+    roof["algorithmic_flops"] = fl
+    roof["avg_launch_us"] = stage_avg_us[dom]
+    roof["peak_source"] = peaks["source"]
+    bfl, bby = block_cost(cfg, touched)
+    ms_step = elapsed_ms / K
+    step_roof = {"flops": bfl, "bytes": bby,
+                 "tensor_frac": bfl / (ms_step * 1e-3) / (peaks["bf16_tflops"] * 1e12),
+                 "hbm_frac": bby / (ms_step * 1e-3) / (peaks["hbm_gbs"] * 1e9)}
+    step_roof["binding_frac"] = max(step_roof["tensor_frac"], step_roof["hbm_frac"])
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = oracle_args(inp)
+        rate, cores, n, dt = cpu_oracle_rate(cfg, host, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} seeded tokens of {cfg.name} (full block per token, fp64), {dt:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) x, N(0,0.02) weights)",
+                "config": {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "E": cfg.E, "k": cfg.k,
+                           "d_ff": cfg.f, "n_shared": cfg.S, "d_ff_shared": cfg.fs, "score_fn": cfg.score_fn,
+                           "norm_topk": cfg.norm_topk, "touched_experts": touched,
+                           "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (
+                               2.0 * cfg.E * 3 * cfg.f * cfg.d / 1e9),
+                           "parallelism": "replicas" if world > 1 else "single GPU"},
+                "roofline": roof, "step_roofline": step_roof,
+                "kernels_us": stage_avg_us, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": K * sum(LAUNCHES_PER_STEP.values()),
+                "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,213 @@
+/*
+ * moe.h - C ABI of libmoe.so, a B200 (sm_100a) mixture-of-experts FFN block.
+ *
+ * The block (archdiff.com architecture-comparison pages; blueprint diagram
+ * "RMSNorm pre-norm -> router -> routed experts top-6-22 of 256-896, SwiGLU ->
+ * shared expert 1-2, always active -> residual add", qwen3-5-vs-deepseek-v4):
+ *
+ *   logits   l = x W_router^T                                   (linear router)
+ *   scores   s = softmax(l) | sigmoid(l) | sqrt(softplus(l))
+ *   pick     the k largest of c = s (+ expert_bias for sigmoid/sqrt-softplus:
+ *            the bias only picks experts), descending, ties to the lower index
+ *   weights  w_j = s_{pick_j}; renormalised over the picks if norm_topk;
+ *            times route_scale
+ *   out      = sum_j w_j SwiGLU_{pick_j}(x) + sum_s SwiGLU_shared_s(x)
+ *            SwiGLU(x) = W_down (SiLU(W_gate x) * (W_up x)), no residual.
+ *
+ * Sources on the pages:
+ *   softmax router "softmax, keep the top k, renormalize, no selection bias":
+ *     qwen3-5-vs-deepseek-v4 component table, Qwen3.5 router cell;
+ *   sqrt-softplus router with selection-only bias, "normalized and scaled by
+ *     2.5": same table, DeepSeek-V4-Pro router cell; sigma form: DeepSeek-V4-Pro
+ *     diagram ("MoE router - sigma / sqrt-softplus - bias balancing");
+ *   SwiGLU experts at full width: qwen3-5-vs-gemma-4 component table, Qwen3.5
+ *     routed-experts cell; shared expert added to the routed sum: same table,
+ *     Qwen3.5 shared-expert cell (ungated, DeepSeek-style, is what is built).
+ *
+ * Conventions for every entry point
+ *   - Tensors are dense, row-major, in device memory unless stated otherwise,
+ *     and owned by the caller.  bf16 = IEEE bfloat16 bit patterns (uint16).
+ *     Weights use the [out, in] layout:
+ *        x [T,d]  W_router [E,d]  W_gate, W_up [E,f,d]  W_down [E,d,f]
+ *        W_shared_gate, W_shared_up [S,fs,d]  W_shared_down [S,d,fs]
+ *   - Every device pointer must be 16-byte aligned; d, f and fs must be
+ *     multiples of 64; 1 <= k <= min(E, 32); 1 <= E <= 2048; 0 <= S <= 8;
+ *     T >= 1.  Violations return an error code and enqueue nothing.
+ *   - `stream` is a cudaStream_t passed as a plain pointer (NULL = legacy
+ *     default stream).  Work is enqueued asynchronously on it; no entry point
+ *     except moe_device_status synchronises the host.
+ *   - The library allocates no device memory and keeps no per-call state: all
+ *     scratch lives in the caller's workspace (size from moe_workspace_bytes),
+ *     which must not be used by two calls that overlap on the GPU.
+ *   - On an error return nothing has been enqueued and the outputs are
+ *     untouched.
+ *   - Kernels never trap.  Every device-side wait is bounded; a wait that runs
+ *     out sets an error word in the workspace, the kernel returns, and
+ *     moe_device_status reports MOE_ERR_DEVICE_TIMEOUT.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK                  0
+#define MOE_ERR_INVALID_ARG    -1   /* null pointer, k<1, k>E, T<1, bad enum ... */
+#define MOE_ERR_UNSUPPORTED    -2   /* d/f/fs not multiples of 64, misaligned pointer, limits, not sm_100 */
+#define MOE_ERR_WORKSPACE      -3   /* workspace missing, misaligned or smaller than moe_workspace_bytes */
+#define MOE_ERR_CUDA           -4   /* a CUDA runtime / driver call or a launch failed */
+#define MOE_ERR_DEVICE_TIMEOUT -5   /* a bounded device-side wait ran out (reported by moe_device_status) */
+
+#define MOE_SCORE_SOFTMAX       0   /* s = softmax(l) over all E experts; expert_bias ignored */
+#define MOE_SCORE_SIGMOID       1   /* s = 1/(1+exp(-l)) */
+#define MOE_SCORE_SQRT_SOFTPLUS 2   /* s = sqrt(log(1+exp(l))) */
+
+typedef void *moe_stream_t;         /* a cudaStream_t */
+
+typedef struct moe_shape {
+    int32_t T;            /* tokens */
+    int32_t d_model;      /* d */
+    int32_t E;            /* routed experts */
+    int32_t k;            /* experts picked per token */
+    int32_t d_ff;         /* f: routed expert hidden width */
+    int32_t n_shared;     /* S: always-active shared experts (0 allowed) */
+    int32_t d_ff_shared;  /* fs: shared expert hidden width (ignored when S == 0) */
+} moe_shape;
+
+/* Library version, MAJOR*10000 + MINOR*100 + PATCH. */
+MOE_API int moe_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+MOE_API const char *moe_status_string(int status);
+
+/* Bytes of workspace that every entry point below needs for this shape
+ * (0 if the shape is invalid).  The workspace must be 256-byte aligned.
+ * Its contents need no initialisation. */
+MOE_API size_t moe_workspace_bytes(const moe_shape *shape);
+
+/* The whole block, steps a1..a7 below in order, on `stream`.
+ *   x, weights: inputs as above.  expert_bias: fp32 [E] or NULL (selection
+ *   only; ignored for MOE_SCORE_SOFTMAX).  W_shared_*: NULL iff S == 0.
+ *   score_fn: MOE_SCORE_*.  norm_topk: 0/1.  route_scale: multiplies the
+ *   combine weights (1.0 = none; DeepSeek-V4-Pro uses 2.5).
+ *   out      [T,d] bf16: the block output, residual-free.
+ *   topk_idx [T,k] int32: picked experts, descending selection key, ties to
+ *            the lower index.
+ *   topk_w   [T,k] fp32: the combine weights actually applied.
+ * Returns MOE_OK or an error code. */
+MOE_API int moe_forward(const moe_shape *shape,
+                const void *x, const void *W_router, const float *expert_bias,
+                const void *W_gate, const void *W_up, const void *W_down,
+                const void *W_shared_gate, const void *W_shared_up, const void *W_shared_down,
+                int score_fn, int norm_topk, float route_scale,
+                void *out, int32_t *topk_idx, float *topk_w,
+                void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* moe_forward with x and the outputs in HOST memory (page-locked memory lets
+ * the copies run asynchronously; pageable memory works but the copies then
+ * synchronise with the host).  The library copies x into the workspace,
+ * runs the block, and copies out / topk_idx / topk_w back, all on `stream`.
+ * Weights and the workspace are device memory.  The host buffers must stay
+ * valid until the stream reaches the end of this call. */
+MOE_API int moe_forward_host(const moe_shape *shape,
+                     const void *x_host, const void *W_router, const float *expert_bias,
+                     const void *W_gate, const void *W_up, const void *W_down,
+                     const void *W_shared_gate, const void *W_shared_up, const void *W_shared_down,
+                     int score_fn, int norm_topk, float route_scale,
+                     void *out_host, int32_t *topk_idx_host, float *topk_w_host,
+                     void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* ---- The steps of moe_forward, callable one by one (same arguments and
+ * rules; each step reads what the previous steps left in the workspace, so
+ * they must be called in this order with the same shape and workspace). ---- */
+
+/* a1 + a2: router GEMM (fp32 accumulate, tcgen05 tensor cores) into fp32
+ * logits in the workspace, then scoring, top-k (bias for selection only) and
+ * optional renormalisation -> topk_idx, topk_w.  Also clears the workspace's
+ * device error word. */
+MOE_API int moe_route(const moe_shape *shape, const void *x, const void *W_router, const float *expert_bias,
+              int score_fn, int norm_topk, float route_scale,
+              int32_t *topk_idx, float *topk_w,
+              void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* a3: per-expert histogram, prefix scan and stable scatter of the (token,
+ * slot) pairs into expert-contiguous rows (tokens ascending inside an expert),
+ * plus the GEMM work lists, all on the device.  topk_idx / topk_w as written
+ * by moe_route (any valid routing may be passed: each row of topk_idx must
+ * hold k distinct experts in [0,E)). */
+MOE_API int moe_permute(const moe_shape *shape, const int32_t *topk_idx, const float *topk_w,
+                void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* a4 + a6 (gate/up half): grouped GEMM over routed rows and the shared
+ * experts' rows in one launch; h = SiLU(x W_gate^T) * (x W_up^T) written as
+ * bf16 into the workspace (fp32 accumulate and epilogue). */
+MOE_API int moe_expert_gate_up(const moe_shape *shape, const void *x,
+                       const void *W_gate, const void *W_up,
+                       const void *W_shared_gate, const void *W_shared_up,
+                       void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* a5 + a6 (down half): grouped GEMM y = w * (h W_down^T) per routed row (w =
+ * its combine weight) and y = h W_shared_down^T per shared row, bf16 into the
+ * workspace. */
+MOE_API int moe_expert_down(const moe_shape *shape, const void *W_down, const void *W_shared_down,
+                    void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* a7: out[t] = sum_s y_shared[s,t] + sum_{j<k} y[row(t,j)], summed in fp32 in
+ * that fixed order and rounded to bf16 once (bitwise reproducible). */
+MOE_API int moe_combine(const moe_shape *shape, void *out,
+                void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* Introspection of the workspace layout, for tests and debugging.  Regions:
+ *   MOE_WS_LOGITS   fp32 [T,E]   router logits (after moe_route)
+ *   MOE_WS_COUNTS   int32 [E]    tokens per expert (after moe_permute)
+ *   MOE_WS_OFFSETS  int32 [E+1]  first row of each expert's segment; segments
+ *                                are padded to 16 rows; [E] = total rows
+ *   MOE_WS_PERM     int32 [rows] token of each routed row (padding rows: 0)
+ *   MOE_WS_ROW_W    fp32 [rows]  combine weight of each routed row (padding: 0)
+ *   MOE_WS_INV      int32 [T,k]  row of each (token, slot)
+ *   MOE_WS_H        bf16 [rows,f]   routed hidden rows (after moe_expert_gate_up)
+ *   MOE_WS_H_SHARED bf16 [S,Tp,fs]  shared hidden rows, Tp = T rounded up to 16
+ *   MOE_WS_Y        bf16 [rows,d]   weighted routed outputs (after moe_expert_down)
+ *   MOE_WS_Y_SHARED bf16 [S,Tp,d]   shared outputs
+ * Writes the region's byte offset in the workspace and its capacity in bytes.
+ * Returns MOE_OK, or MOE_ERR_INVALID_ARG for a bad shape, region or pointer. */
+#define MOE_WS_LOGITS   0
+#define MOE_WS_COUNTS   1
+#define MOE_WS_OFFSETS  2
+#define MOE_WS_PERM     3
+#define MOE_WS_ROW_W    4
+#define MOE_WS_INV      5
+#define MOE_WS_H        6
+#define MOE_WS_H_SHARED 7
+#define MOE_WS_Y        8
+#define MOE_WS_Y_SHARED 9
+MOE_API int moe_workspace_region(const moe_shape *shape, int region, size_t *offset, size_t *bytes);
+
+/* Synchronises `stream`, then returns MOE_ERR_DEVICE_TIMEOUT if a kernel of a
+ * call on this workspace (since the last moe_route) gave up a bounded wait,
+ * MOE_ERR_CUDA if the stream reports an error, else MOE_OK. */
+MOE_API int moe_device_status(const void *workspace, moe_stream_t stream);
+
+/* Self-test of the bounded-wait machinery: launches one block that waits on a
+ * shared-memory barrier which nothing ever completes, for at most timeout_ns
+ * nanoseconds (clamped to 1 ms .. 1 s), then records the timeout in the
+ * workspace's error word and returns.  moe_device_status then reports
+ * MOE_ERR_DEVICE_TIMEOUT and the context stays usable. */
+MOE_API int moe_debug_wait_timeout(void *workspace, size_t workspace_bytes, uint64_t timeout_ns,
+                           moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

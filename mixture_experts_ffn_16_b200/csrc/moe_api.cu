@@ -1,0 +1,496 @@
+// moe_api.cu - the C ABI of libmoe.so (declared in include/moe.h): argument
+// checks, the workspace plan, TMA tensor maps, and the launch sequence
+//   router GEMM -> top-k -> permute (count, scan, scatter) ->
+//   gate/up GEMM -> down GEMM -> combine
+// on the caller's stream.  No host synchronisation, no device allocation.
+#include <cmath>
+#include <cstring>
+
+#include "moe_internal.h"
+#include "moe_ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// Weight tensor [G, rows, K] bf16 -> tiles of 128 rows x 64 K, 128-byte swizzle.
+bool map_weights(CUtensorMap* m, const void* ptr, int K, int rows, int G) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(G)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, static_cast<cuuint64_t>(K) * 2 * rows};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(kTileRows), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-gather source [rows, K] bf16: box of one row x 64 K, 128-byte swizzle.
+bool map_rows(CUtensorMap* m, const void* ptr, int K, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), 1};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int pick_nmax(double rows_per_expert) {
+  int n = 16;
+  while (n < 256 && n < rows_per_expert * 1.25) n *= 2;
+  return n;
+}
+
+int check_ws(const Plan& p, const void* ws, size_t bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < p.total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+int check_device(DeviceInfo* di) {
+  if (device_info(di) != MOE_OK || !di->ok) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ---- the steps, after validation ----
+
+int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_router, const float* bias,
+              int score_fn, int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w, char* ws,
+              cudaStream_t st) {
+  if (cudaMemsetAsync(ws + p.err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+  GemmParams g;
+  std::memset(&g, 0, sizeof g);
+  if (!map_weights(&g.mapA[0], W_router, p.d, p.E, 1) || !map_rows(&g.mapB[0], x, p.d, p.T))
+    return MOE_ERR_CUDA;
+  g.mapA[1] = g.mapA[2] = g.mapA[3] = g.mapA[0];
+  g.mapB[1] = g.mapB[0];
+  g.num_units_host = p.router_units;
+  g.out_r = ws + p.logits;
+  g.err = reinterpret_cast<uint32_t*>(ws + p.err);
+  g.T = p.T; g.Tp = p.Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
+  g.nmax = p.nmax_r;
+  g.router_nwb = p.nwbE;
+  g.timeout_ns = kWaitTimeoutNs;
+  int stages = 0;
+  const size_t smem = gemm_smem_bytes(kModeRouter, p.nmax_r, &stages);
+  g.stages = stages;
+  g.nbuf = (p.nmax_r <= 256) ? 2 : 1;
+  const int grid = p.router_units < di.sms ? p.router_units : di.sms;
+  int rc = launch_gemm(kModeRouter, g, grid, smem, st);
+  if (rc != MOE_OK) return rc;
+  return launch_topk(reinterpret_cast<const float*>(ws + p.logits), bias, p.T, p.E, p.k, score_fn, norm_topk,
+                     route_scale, topk_idx, topk_w, st);
+}
+
+int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* Wg, const void* Wu,
+                const void* Wsg, const void* Wsu, char* ws, cudaStream_t st) {
+  GemmParams g;
+  std::memset(&g, 0, sizeof g);
+  if (!map_weights(&g.mapA[0], Wg, p.d, p.f, p.E) || !map_weights(&g.mapA[1], Wu, p.d, p.f, p.E) ||
+      !map_rows(&g.mapB[0], x, p.d, p.T))
+    return MOE_ERR_CUDA;
+  if (p.S > 0) {
+    if (!map_weights(&g.mapA[2], Wsg, p.d, p.fs, p.S) || !map_weights(&g.mapA[3], Wsu, p.d, p.fs, p.S))
+      return MOE_ERR_CUDA;
+  } else {
+    g.mapA[2] = g.mapA[0];
+    g.mapA[3] = g.mapA[1];
+  }
+  g.mapB[1] = g.mapB[0];
+  g.units = reinterpret_cast<const int4*>(ws + p.units1);
+  g.num_units_dev = reinterpret_cast<const int*>(ws + p.nunits);
+  g.perm = reinterpret_cast<const int*>(ws + p.perm);
+  g.out_r = ws + p.Hr;
+  g.out_s = ws + p.Hs;
+  g.err = reinterpret_cast<uint32_t*>(ws + p.err);
+  g.T = p.T; g.Tp = p.Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
+  g.nmax = p.nmax1;
+  g.timeout_ns = kWaitTimeoutNs;
+  int stages = 0;
+  const size_t smem = gemm_smem_bytes(kModeGateUp, p.nmax1, &stages);
+  g.stages = stages;
+  g.nbuf = (2 * p.nmax1 <= 256) ? 2 : 1;
+  return launch_gemm(kModeGateUp, g, di.sms, smem, st);
+}
+
+int run_down(const Plan& p, const DeviceInfo& di, const void* Wd, const void* Wsd, char* ws, cudaStream_t st) {
+  GemmParams g;
+  std::memset(&g, 0, sizeof g);
+  if (!map_weights(&g.mapA[0], Wd, p.f, p.d, p.E) || !map_rows(&g.mapB[0], ws + p.Hr, p.f, p.Rcap))
+    return MOE_ERR_CUDA;
+  if (p.S > 0) {
+    if (!map_weights(&g.mapA[2], Wsd, p.fs, p.d, p.S) || !map_rows(&g.mapB[1], ws + p.Hs, p.fs, p.S * p.Tp))
+      return MOE_ERR_CUDA;
+  } else {
+    g.mapA[2] = g.mapA[0];
+    g.mapB[1] = g.mapB[0];
+  }
+  g.mapA[1] = g.mapA[0];
+  g.mapA[3] = g.mapA[2];
+  g.units = reinterpret_cast<const int4*>(ws + p.units2);
+  g.num_units_dev = reinterpret_cast<const int*>(ws + p.nunits) + 1;
+  g.roww = reinterpret_cast<const float*>(ws + p.roww);
+  g.out_r = ws + p.Yr;
+  g.out_s = ws + p.Ys;
+  g.err = reinterpret_cast<uint32_t*>(ws + p.err);
+  g.T = p.T; g.Tp = p.Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
+  g.nmax = p.nmax2;
+  g.timeout_ns = kWaitTimeoutNs;
+  int stages = 0;
+  const size_t smem = gemm_smem_bytes(kModeDown, p.nmax2, &stages);
+  g.stages = stages;
+  g.nbuf = (p.nmax2 <= 256) ? 2 : 1;
+  return launch_gemm(kModeDown, g, di.sms, smem, st);
+}
+
+int check_route_args(const void* x, const void* W_router, const float* bias, int score_fn, int norm_topk,
+                     float route_scale, const void* topk_idx, const void* topk_w) {
+  if (!x || !W_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (score_fn < MOE_SCORE_SOFTMAX || score_fn > MOE_SCORE_SQRT_SOFTPLUS) return MOE_ERR_INVALID_ARG;
+  if (norm_topk != 0 && norm_topk != 1) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(route_scale)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W_router) || !aligned16(topk_idx) || !aligned16(topk_w) ||
+      (bias && !aligned16(bias)))
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+int check_expert_args(const Plan& p, const void* Wg, const void* Wu, const void* Wd, const void* Wsg,
+                      const void* Wsu, const void* Wsd) {
+  if (!Wg || !Wu || !Wd) return MOE_ERR_INVALID_ARG;
+  if (p.S > 0 && (!Wsg || !Wsu || !Wsd)) return MOE_ERR_INVALID_ARG;
+  if (p.S == 0 && (Wsg || Wsu || Wsd)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(Wg) || !aligned16(Wu) || !aligned16(Wd)) return MOE_ERR_UNSUPPORTED;
+  if (p.S > 0 && (!aligned16(Wsg) || !aligned16(Wsu) || !aligned16(Wsd))) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+int forward_impl(const Plan& p, const DeviceInfo& di, const void* x, const void* W_router,
+                 const float* expert_bias, const void* W_gate, const void* W_up, const void* W_down,
+                 const void* W_shared_gate, const void* W_shared_up, const void* W_shared_down, int score_fn,
+                 int norm_topk, float route_scale, void* out, int32_t* topk_idx, float* topk_w, char* ws,
+                 cudaStream_t st) {
+  int rc = run_route(p, di, x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w, ws, st);
+  if (rc == MOE_OK) rc = launch_permute(p, topk_idx, topk_w, ws, st);
+  if (rc == MOE_OK) rc = run_gate_up(p, di, x, W_gate, W_up, W_shared_gate, W_shared_up, ws, st);
+  if (rc == MOE_OK) rc = run_down(p, di, W_down, W_shared_down, ws, st);
+  if (rc == MOE_OK) rc = launch_combine(p, out, ws, st);
+  return rc;
+}
+
+}  // namespace
+
+int make_plan(const moe_shape* s, Plan* p) {
+  if (!s || !p) return MOE_ERR_INVALID_ARG;
+  const int T = s->T, d = s->d_model, E = s->E, k = s->k, f = s->d_ff, S = s->n_shared;
+  const int fs = S > 0 ? s->d_ff_shared : 0;
+  if (T < 1 || E < 1 || k < 1 || k > E || d < 1 || f < 1 || S < 0) return MOE_ERR_INVALID_ARG;
+  if (S > 0 && fs < 1) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxE || k > kMaxK || S > kMaxShared) return MOE_ERR_UNSUPPORTED;
+  if (d % 64 || f % 64 || (S > 0 && fs % 64)) return MOE_ERR_UNSUPPORTED;
+  if (T > (1 << 22) || d > (1 << 16) || f > (1 << 16) || fs > (1 << 16)) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * k + static_cast<long long>(E) * kRowPad > (1ll << 30)) return MOE_ERR_UNSUPPORTED;
+  Plan q;
+  std::memset(&q, 0, sizeof q);
+  q.T = T; q.d = d; q.E = E; q.k = k; q.f = f; q.S = S; q.fs = fs;
+  q.Tp = ceil_div(T, kRowPad) * kRowPad;
+  q.Rcap = ceil_div(T * k + E * (kRowPad - 1), kRowPad) * kRowPad;
+  q.nb = ceil_div(T, kPermBlock);
+  q.nwbE = ceil_div(E, kTileRows);
+  q.nwb1 = ceil_div(f, kTileRows);
+  q.nwb1s = S > 0 ? ceil_div(fs, kTileRows) : 0;
+  q.nwb2 = ceil_div(d, kTileRows);
+  const double rows_per_expert = static_cast<double>(T) * k / E;
+  q.nmax1 = pick_nmax(rows_per_expert);
+  q.nmax2 = q.nmax1;
+  // Router: the widest token run that still gives every SM of a B200 a unit.
+  q.nmax_r = 16;
+  for (int n = 256; n >= 16; n >>= 1) {
+    if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, n) >= 148) {
+      q.nmax_r = n;
+      break;
+    }
+  }
+  q.router_units = q.nwbE * ceil_div(q.Tp, q.nmax_r);
+  q.shared_units1 = S * q.nwb1s * ceil_div(q.Tp, q.nmax1);
+  q.shared_units2 = S * q.nwb2 * ceil_div(q.Tp, q.nmax2);
+  q.U1cap = q.shared_units1 + q.nwb1 * (q.Rcap / q.nmax1 + E);
+  q.U2cap = q.shared_units2 + q.nwb2 * (q.Rcap / q.nmax2 + E);
+
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  q.err = take(16);
+  q.nunits = take(16);
+  q.logits = take(static_cast<size_t>(T) * E * 4);
+  q.blkcnt = take(static_cast<size_t>(q.nb) * E * 4);
+  q.counts = take(static_cast<size_t>(E) * 4);
+  q.roff = take(static_cast<size_t>(E + 1) * 4);
+  q.perm = take(static_cast<size_t>(q.Rcap) * 4);
+  q.roww = take(static_cast<size_t>(q.Rcap) * 4);
+  q.inv = take(static_cast<size_t>(T) * k * 4);
+  q.units1 = take(static_cast<size_t>(q.U1cap) * 16);
+  q.units2 = take(static_cast<size_t>(q.U2cap) * 16);
+  q.Hr = take(static_cast<size_t>(q.Rcap) * f * 2);
+  q.Hs = take(static_cast<size_t>(S) * q.Tp * (fs > 0 ? fs : 0) * 2);
+  q.Yr = take(static_cast<size_t>(q.Rcap) * d * 2);
+  q.Ys = take(static_cast<size_t>(S) * q.Tp * d * 2);
+  q.xstage = take(static_cast<size_t>(T) * d * 2);
+  q.ostage = take(static_cast<size_t>(T) * d * 2);
+  q.istage = take(static_cast<size_t>(T) * k * 4);
+  q.wstage = take(static_cast<size_t>(T) * k * 4);
+  q.total = off;
+  *p = q;
+  return MOE_OK;
+}
+
+int device_info(DeviceInfo* info) {
+  static DeviceInfo cache[64];
+  static int have[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  if (!have[dev]) {
+    DeviceInfo d;
+    std::memset(&d, 0, sizeof d);
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    d.ok = (major == 10 && d.max_smem_optin >= 232448 && encode_fn() != nullptr) ? 1 : 0;
+    cache[dev] = d;
+    have[dev] = 1;
+  }
+  *info = cache[dev];
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_version(void) { return 100; }
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: unsupported shape, alignment or device";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA call or kernel launch failed";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a bounded device-side wait ran out";
+    default: return "unknown status";
+  }
+}
+
+size_t moe_workspace_bytes(const moe_shape* shape) {
+  Plan p;
+  if (make_plan(shape, &p) != MOE_OK) return 0;
+  return p.total;
+}
+
+int moe_route(const moe_shape* shape, const void* x, const void* W_router, const float* expert_bias,
+              int score_fn, int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w, void* workspace,
+              size_t workspace_bytes, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_route_args(x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w)) != MOE_OK)
+    return rc;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return run_route(p, di, x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w,
+                   static_cast<char*>(workspace), as_stream(stream));
+}
+
+int moe_permute(const moe_shape* shape, const int32_t* topk_idx, const float* topk_w, void* workspace,
+                size_t workspace_bytes, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if (!topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(topk_idx) || !aligned16(topk_w)) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return launch_permute(p, topk_idx, topk_w, static_cast<char*>(workspace), as_stream(stream));
+}
+
+int moe_expert_gate_up(const moe_shape* shape, const void* x, const void* W_gate, const void* W_up,
+                       const void* W_shared_gate, const void* W_shared_up, void* workspace, size_t workspace_bytes,
+                       moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if (!x || !W_gate || !W_up) return MOE_ERR_INVALID_ARG;
+  if (p.S > 0 && (!W_shared_gate || !W_shared_up)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W_gate) || !aligned16(W_up) ||
+      (p.S > 0 && (!aligned16(W_shared_gate) || !aligned16(W_shared_up))))
+    return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return run_gate_up(p, di, x, W_gate, W_up, W_shared_gate, W_shared_up, static_cast<char*>(workspace),
+                     as_stream(stream));
+}
+
+int moe_expert_down(const moe_shape* shape, const void* W_down, const void* W_shared_down, void* workspace,
+                    size_t workspace_bytes, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if (!W_down || (p.S > 0 && !W_shared_down)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(W_down) || (p.S > 0 && !aligned16(W_shared_down))) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return run_down(p, di, W_down, W_shared_down, static_cast<char*>(workspace), as_stream(stream));
+}
+
+int moe_combine(const moe_shape* shape, void* out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if (!out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out)) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return launch_combine(p, out, static_cast<const char*>(workspace), as_stream(stream));
+}
+
+int moe_forward(const moe_shape* shape, const void* x, const void* W_router, const float* expert_bias,
+                const void* W_gate, const void* W_up, const void* W_down, const void* W_shared_gate,
+                const void* W_shared_up, const void* W_shared_down, int score_fn, int norm_topk, float route_scale,
+                void* out, int32_t* topk_idx, float* topk_w, void* workspace, size_t workspace_bytes,
+                moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_route_args(x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w)) != MOE_OK)
+    return rc;
+  if ((rc = check_expert_args(p, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down)) != MOE_OK)
+    return rc;
+  if (!out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out)) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return forward_impl(p, di, x, W_router, expert_bias, W_gate, W_up, W_down, W_shared_gate, W_shared_up,
+                      W_shared_down, score_fn, norm_topk, route_scale, out, topk_idx, topk_w,
+                      static_cast<char*>(workspace), as_stream(stream));
+}
+
+int moe_forward_host(const moe_shape* shape, const void* x_host, const void* W_router, const float* expert_bias,
+                     const void* W_gate, const void* W_up, const void* W_down, const void* W_shared_gate,
+                     const void* W_shared_up, const void* W_shared_down, int score_fn, int norm_topk,
+                     float route_scale, void* out_host, int32_t* topk_idx_host, float* topk_w_host,
+                     void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if (!x_host || !out_host || !topk_idx_host || !topk_w_host) return MOE_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  void* xd = ws + p.xstage;
+  void* od = ws + p.ostage;
+  int32_t* id = reinterpret_cast<int32_t*>(ws + p.istage);
+  float* wd = reinterpret_cast<float*>(ws + p.wstage);
+  if ((rc = check_route_args(xd, W_router, expert_bias, score_fn, norm_topk, route_scale, id, wd)) != MOE_OK)
+    return rc;
+  if ((rc = check_expert_args(p, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down)) != MOE_OK)
+    return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  cudaStream_t st = as_stream(stream);
+  const size_t xbytes = static_cast<size_t>(p.T) * p.d * 2;
+  const size_t tkbytes = static_cast<size_t>(p.T) * p.k * 4;
+  if (cudaMemcpyAsync(xd, x_host, xbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
+  rc = forward_impl(p, di, xd, W_router, expert_bias, W_gate, W_up, W_down, W_shared_gate, W_shared_up,
+                    W_shared_down, score_fn, norm_topk, route_scale, od, id, wd, ws, st);
+  if (rc != MOE_OK) return rc;
+  if (cudaMemcpyAsync(out_host, od, xbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(topk_idx_host, id, tkbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(topk_w_host, wd, tkbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_workspace_region(const moe_shape* shape, int region, size_t* offset, size_t* bytes) {
+  Plan p;
+  if (!offset || !bytes) return MOE_ERR_INVALID_ARG;
+  if (make_plan(shape, &p) != MOE_OK) return MOE_ERR_INVALID_ARG;
+  const size_t T = p.T, E = p.E, k = p.k, R = p.Rcap, S = p.S, Tp = p.Tp;
+  switch (region) {
+    case MOE_WS_LOGITS: *offset = p.logits; *bytes = T * E * 4; break;
+    case MOE_WS_COUNTS: *offset = p.counts; *bytes = E * 4; break;
+    case MOE_WS_OFFSETS: *offset = p.roff; *bytes = (E + 1) * 4; break;
+    case MOE_WS_PERM: *offset = p.perm; *bytes = R * 4; break;
+    case MOE_WS_ROW_W: *offset = p.roww; *bytes = R * 4; break;
+    case MOE_WS_INV: *offset = p.inv; *bytes = T * k * 4; break;
+    case MOE_WS_H: *offset = p.Hr; *bytes = R * p.f * 2; break;
+    case MOE_WS_H_SHARED: *offset = p.Hs; *bytes = S * Tp * p.fs * 2; break;
+    case MOE_WS_Y: *offset = p.Yr; *bytes = R * p.d * 2; break;
+    case MOE_WS_Y_SHARED: *offset = p.Ys; *bytes = S * Tp * p.d * 2; break;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+int moe_device_status(const void* workspace, moe_stream_t stream) {
+  if (!workspace) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word & kDevErrTimeout) return MOE_ERR_DEVICE_TIMEOUT;
+  if (word & kDevErrBadRouting) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+int moe_debug_wait_timeout(void* workspace, size_t workspace_bytes, uint64_t timeout_ns, moe_stream_t stream) {
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < 256)
+    return MOE_ERR_WORKSPACE;
+  DeviceInfo di;
+  int rc = check_device(&di);
+  if (rc != MOE_OK) return rc;
+  if (timeout_ns < 1000000ull) timeout_ns = 1000000ull;
+  if (timeout_ns > 1000000000ull) timeout_ns = 1000000000ull;
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), as_stream(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_wait_timeout(reinterpret_cast<uint32_t*>(workspace), timeout_ns, as_stream(stream));
+}
+
+}  // extern "C"

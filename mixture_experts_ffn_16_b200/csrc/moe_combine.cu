@@ -1,0 +1,96 @@
+// moe_combine.cu - gate-weighted combine (step a7) and the bounded-wait
+// self-test kernel.
+//
+// out[t, :] = sum_{s<S} Y_shared[s, t, :] + sum_{j<k} Y[inv[t, j], :]
+// The routed rows already carry their combine weight (applied in fp32 by the
+// down GEMM before rounding).  Each thread owns 8 consecutive features of one
+// token, adds the S + k bf16 rows in that fixed order in fp32 and rounds once,
+// so the result is bitwise reproducible and independent of the row layout.
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+#include "moe_ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kCombineThreads = 256;
+
+__device__ __forceinline__ void add8(float (&acc)[8], const uint4 v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    acc[2 * i] += f.x;
+    acc[2 * i + 1] += f.y;
+  }
+}
+
+__global__ void __launch_bounds__(kCombineThreads)
+combine_kernel(const __nv_bfloat16* __restrict__ Yr, const __nv_bfloat16* __restrict__ Ys,
+               const int32_t* __restrict__ inv, __nv_bfloat16* __restrict__ out, int T, int d, int k,
+               int S, int Tp) {
+  const int chunks = d >> 3;
+  const size_t total = static_cast<size_t>(T) * chunks;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(i / chunks);
+    const int c = static_cast<int>(i - static_cast<size_t>(t) * chunks);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < S; ++s) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+          Ys + (static_cast<size_t>(s) * Tp + t) * d + static_cast<size_t>(c) * 8));
+      add8(acc, v);
+    }
+    const int32_t* it = inv + static_cast<size_t>(t) * k;
+    for (int j = 0; j < k; ++j) {
+      const int row = __ldg(it + j);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(Yr + static_cast<size_t>(row) * d +
+                                                           static_cast<size_t>(c) * 8));
+      add8(acc, v);
+    }
+    uint4 o;
+    __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) oh[q] = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+    *reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * d + static_cast<size_t>(c) * 8) = o;
+  }
+}
+
+// Waits on a barrier that nothing completes, for at most timeout_ns, then
+// records the timeout.  Used to test the bounded-wait path without a hang.
+__global__ void wait_timeout_kernel(uint32_t* err, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_wait(&bar, 0, &abort_flag, err, timeout_ns);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+int launch_combine(const Plan& p, void* out, const char* ws, cudaStream_t st) {
+  const size_t total = static_cast<size_t>(p.T) * (p.d / 8);
+  size_t blocks = (total + kCombineThreads - 1) / kCombineThreads;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  combine_kernel<<<static_cast<int>(blocks), kCombineThreads, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(ws + p.Yr), reinterpret_cast<const __nv_bfloat16*>(ws + p.Ys),
+      reinterpret_cast<const int32_t*>(ws + p.inv), reinterpret_cast<__nv_bfloat16*>(out), p.T, p.d,
+      p.k, p.S, p.Tp);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_wait_timeout(uint32_t* err, uint64_t timeout_ns, cudaStream_t st) {
+  wait_timeout_kernel<<<1, 32, 0, st>>>(err, timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

@@ -1,0 +1,398 @@
+// moe_gemm.cu - the tensor-core GEMMs of the MoE block on sm_100a:
+//
+//   router  : logits[t, e]   = x[t,:] . W_router[e,:]                      (fp32 out)
+//   gate/up : H[r, j]        = SiLU(x[tok(r),:] . Wg[e,j,:]) * (x[tok(r),:] . Wu[e,j,:])
+//   down    : Y[r, m]        = w(r) * (H[r,:] . Wd[e,m,:])
+//
+// One persistent, warp-specialised kernel template serves all three.  A work
+// unit is (group g, 128-row block of the weight matrix, a run of n <= nmax
+// consecutive rows of the group's row segment).  The GEMM is "swap-AB": the
+// 128 weight rows are the MMA's M side and the unit's tokens its N side
+// (n a multiple of 16), so an expert with few tokens costs n/16 MMA columns,
+// not a padded 128-row tile.
+//
+//   warp 0      TMA producer: weight tiles by 3-D tiled loads, token rows by
+//               tile::gather4 loads (4 arbitrary rows per instruction, no
+//               permuted copy of x is ever made), into a ring of stages.
+//   warp 1      TMEM owner and single-thread tcgen05.mma issuer; fp32
+//               accumulators in tensor memory (gate and up side by side for
+//               the gate/up GEMM), double-buffered when they fit.
+//   warps 2..5  epilogue: tcgen05.ld -> fp32 math (SiLU*, weight scale) ->
+//               bf16 -> transpose through shared memory -> 16-byte stores of
+//               whole row segments.
+//
+// All waits are bounded (see mbar_wait); a block that gives up records the
+// timeout in the workspace error word, drains its own copies and MMAs, frees
+// its tensor memory and returns.
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+#include "moe_ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kATileBytes = kTileRows * 128;   // 128 weight rows x 64 bf16
+constexpr int kEpiStageBytes = 2048;                 // per epilogue warp
+constexpr int kMaxStages = 8;
+constexpr int kSmemAlign = 1024;
+constexpr int kSmemTail = 256;                       // barriers, TMEM slot, abort flag
+
+struct Unit {
+  int g, wb, row0, n;
+};
+
+template <int MODE>
+__device__ __forceinline__ Unit get_unit(const GemmParams& p, int u) {
+  Unit un;
+  if (MODE == kModeRouter) {
+    const int chunk = u / p.router_nwb;
+    un.g = 0;
+    un.wb = u - chunk * p.router_nwb;
+    un.row0 = chunk * p.nmax;
+    un.n = min(p.nmax, p.Tp - un.row0);
+  } else {
+    const int4 v = __ldg(p.units + u);
+    un.g = v.x;
+    un.wb = v.y;
+    un.row0 = v.z;
+    un.n = v.w;
+  }
+  return un;
+}
+
+// Bounded wait that ignores the abort flag: used only to drain work this block
+// itself put in flight before it leaves.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (global_timer_ns() - t0 > timeout_ns) return;
+  }
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1) moe_gemm_kernel(const __grid_constant__ GemmParams p) {
+  constexpr int NA = (MODE == kModeGateUp) ? 2 : 1;   // A operands (accumulators) per unit
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + (kSmemAlign - 1)) & ~static_cast<uintptr_t>(kSmemAlign - 1));
+  const int nmax = p.nmax;
+  const int S = p.stages;
+  const uint32_t stage_bytes = NA * kATileBytes + static_cast<uint32_t>(nmax) * 128u;
+  uint8_t* epi = smem + static_cast<size_t>(S) * stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi + 4 * kEpiStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < 2 * NA; ++i) prefetch_tensormap(&p.mapA[i]);
+    prefetch_tensormap(&p.mapB[0]);
+    if (MODE == kModeDown) prefetch_tensormap(&p.mapB[1]);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_units = (MODE == kModeRouter) ? p.num_units_host : *p.num_units_dev;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      const Unit un = get_unit<MODE>(p, u);
+      const bool sh = (MODE != kModeRouter) && un.g >= p.E;
+      const int sidx = sh ? un.g - p.E : 0;
+      const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
+      const int KB = K / kTileK;
+      const CUtensorMap* mA = &p.mapA[sh ? 2 : 0];
+      const CUtensorMap* mB = &p.mapB[(MODE == kModeDown && sh) ? 1 : 0];
+      const int a_c2 = (MODE == kModeRouter) ? 0 : (sh ? sidx : un.g);
+      // Source rows of this lane's gathers: quads q = lane and lane + 32.
+      int rows[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int i = 4 * (lane + 32 * j) + r;
+          int src = 0;
+          if (i < un.n) {
+            if (MODE == kModeRouter) {
+              src = min(un.row0 + i, p.T - 1);
+            } else if (MODE == kModeGateUp) {
+              src = sh ? min(un.row0 + i, p.T - 1) : __ldg(p.perm + un.row0 + i);
+            } else {
+              src = sh ? sidx * p.Tp + un.row0 + i : un.row0 + i;
+            }
+          }
+          rows[j][r] = src;
+        }
+      }
+      const uint32_t tx_bytes = NA * kATileBytes + static_cast<uint32_t>(un.n) * 128u;
+      for (int kb = 0; kb < KB; ++kb) {
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          ok = false;
+          break;
+        }
+        const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+        const uint32_t fb = smem_u32(&full[stage]);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], tx_bytes);
+#pragma unroll
+          for (int a = 0; a < NA; ++a)
+            tma_load_3d(sbase + a * kATileBytes, mA + a, fb, kb * kTileK, un.wb * kTileRows, a_c2);
+        }
+        __syncwarp();
+        const uint32_t bbase = sbase + NA * kATileBytes;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int qd = lane + 32 * j;
+          if (4 * qd < un.n)
+            tma_gather4(bbase + qd * 512u, mB, fb, kb * kTileK, rows[j][0], rows[j][1], rows[j][2],
+                        rows[j][3]);
+        }
+        ++issued;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // Leave no copy in flight: the last min(S, issued) stages armed.
+    if (lane == 0) {
+      const uint32_t outstanding = issued < static_cast<uint32_t>(S) ? issued : static_cast<uint32_t>(S);
+      for (uint32_t i = 1; i <= outstanding; ++i) {
+        const uint32_t I = issued - i;
+        mbar_wait_drain(&full[I % S], (I / S) & 1u, p.timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t ucount = 0;
+      bool any = false;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const Unit un = get_unit<MODE>(p, u);
+        const bool sh = (MODE != kModeRouter) && un.g >= p.E;
+        const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
+        const int KB = K / kTileK;
+        const int buf = static_cast<int>(ucount % static_cast<uint32_t>(p.nbuf));
+        const uint32_t bpar = (ucount / static_cast<uint32_t>(p.nbuf)) & 1u;
+        if (!mbar_wait(&tempty[buf], bpar ^ 1u, abort_flag, p.err, p.timeout_ns)) break;
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16_f32(kTileRows, un.n);
+        const uint32_t dcol = tmem_base + static_cast<uint32_t>(buf * NA * nmax);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+          const uint64_t bdesc = sw128_kmajor_desc(sbase + NA * kATileBytes);
+          uint64_t adesc[NA];
+#pragma unroll
+          for (int a = 0; a < NA; ++a) adesc[a] = sw128_kmajor_desc(sbase + a * kATileBytes);
+#pragma unroll
+          for (int ks = 0; ks < kTileK / 16; ++ks) {
+#pragma unroll
+            for (int a = 0; a < NA; ++a)
+              tc_mma_bf16(dcol + static_cast<uint32_t>(a * nmax), adesc[a] + 2u * ks, bdesc + 2u * ks,
+                          idesc, (kb | ks) != 0 ? 1u : 0u);
+          }
+          any = true;
+          tc_commit(&empty[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[buf]);
+        ++ucount;
+      }
+      // Leave no MMA in flight.
+      if (any) {
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                       // TMEM lane quarter this warp may read
+    uint8_t* stg = epi + (warp - 2) * kEpiStageBytes;
+    uint32_t ucount = 0;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      const Unit un = get_unit<MODE>(p, u);
+      const bool sh = (MODE != kModeRouter) && un.g >= p.E;
+      const int sidx = sh ? un.g - p.E : 0;
+      const int buf = static_cast<int>(ucount % static_cast<uint32_t>(p.nbuf));
+      const uint32_t bpar = (ucount / static_cast<uint32_t>(p.nbuf)) & 1u;
+      int got = 1;
+      if (lane == 0) got = mbar_wait(&tfull[buf], bpar, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) break;
+      tc_fence_after();
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * NA * nmax);
+      const int feat0 = un.wb * kTileRows + 32 * q;   // first weight row of this warp
+      const int wrows = (MODE == kModeRouter) ? p.E : (MODE == kModeGateUp ? (sh ? p.fs : p.f) : p.d);
+      if (feat0 < wrows) {
+        for (int c0 = 0; c0 < un.n; c0 += 16) {
+          uint32_t acc0[16], acc1[16];
+          tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c0), acc0);
+          if (NA == 2) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c0), acc1);
+          tmem_ld_wait();
+          if (MODE == kModeRouter) {
+            float* sf = reinterpret_cast<float*>(stg);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sf[i * 32 + lane] = __uint_as_float(acc0[i]);
+            __syncwarp();
+#pragma unroll
+            for (int rep = 0; rep < 4; ++rep) {
+              const int c = lane + 32 * rep;
+              const int tok = c >> 3, part = c & 7;
+              const int t = un.row0 + c0 + tok;
+              const int e = feat0 + part * 4;
+              if (t < p.T) {
+                float* dst = reinterpret_cast<float*>(p.out_r) + static_cast<size_t>(t) * p.E + e;
+                const float4 v = *reinterpret_cast<const float4*>(sf + tok * 32 + part * 4);
+                if ((p.E & 3) == 0 && e + 3 < p.E) {
+                  *reinterpret_cast<float4*>(dst) = v;
+                } else {
+                  if (e + 0 < p.E) dst[0] = v.x;
+                  if (e + 1 < p.E) dst[1] = v.y;
+                  if (e + 2 < p.E) dst[2] = v.z;
+                  if (e + 3 < p.E) dst[3] = v.w;
+                }
+              }
+            }
+            __syncwarp();
+          } else {
+            __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
+            if (MODE == kModeGateUp) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float g = __uint_as_float(acc0[i]);
+                const float v = __uint_as_float(acc1[i]);
+                sb[i * 32 + lane] = __float2bfloat16_rn(silu_f(g) * v);
+              }
+            } else {
+              float wl = 1.0f;
+              if (!sh && lane < 16) wl = __ldg(p.roww + un.row0 + c0 + lane);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float w = __shfl_sync(0xffffffffu, wl, i);
+                sb[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(acc0[i]) * w);
+              }
+            }
+            __syncwarp();
+            const int ld = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
+            __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(sh ? p.out_s : p.out_r);
+            const size_t rbase = sh ? static_cast<size_t>(sidx) * p.Tp : 0;
+#pragma unroll
+            for (int rep = 0; rep < 2; ++rep) {
+              const int c = lane + 32 * rep;
+              const int tok = c >> 2, part = c & 3;
+              const uint4 v = *reinterpret_cast<const uint4*>(stg + tok * 64 + part * 16);
+              const size_t row = rbase + static_cast<size_t>(un.row0 + c0 + tok);
+              *reinterpret_cast<uint4*>(outp + row * ld + feat0 + part * 8) = v;
+            }
+            __syncwarp();
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      ++ucount;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+size_t gemm_smem_bytes(int mode, int nmax, int* stages) {
+  const int NA = (mode == kModeGateUp) ? 2 : 1;
+  const size_t stage_bytes = NA * static_cast<size_t>(kATileBytes) + static_cast<size_t>(nmax) * 128;
+  const size_t fixed = kSmemAlign + 4 * kEpiStageBytes + kSmemTail;
+  const size_t budget = 232448;   // sm_100 opt-in maximum per block
+  int s = static_cast<int>((budget - fixed) / stage_bytes);
+  if (s > kMaxStages) s = kMaxStages;
+  if (stages) *stages = s;
+  return fixed + static_cast<size_t>(s) * stage_bytes;
+}
+
+template <int MODE>
+static int launch_mode(const GemmParams& prm, int grid, size_t smem, cudaStream_t st) {
+  static int configured[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  if (configured[dev] < static_cast<int>(smem)) {
+    if (cudaFuncSetAttribute(moe_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured[dev] = static_cast<int>(smem);
+  }
+  moe_gemm_kernel<MODE><<<grid, kThreads, smem, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st) {
+  if (grid < 1) return MOE_OK;
+  switch (mode) {
+    case kModeRouter: return launch_mode<kModeRouter>(prm, grid, smem, st);
+    case kModeGateUp: return launch_mode<kModeGateUp>(prm, grid, smem, st);
+    case kModeDown: return launch_mode<kModeDown>(prm, grid, smem, st);
+    default: return MOE_ERR_INVALID_ARG;
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,92 @@
+// moe_internal.h - host-side plan of one call: workspace carve-up, tiling
+// choices and the launchers of each kernel.  Shared by the .cu files of
+// libmoe.so only.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kMaxE = 2048;
+constexpr int kMaxK = 32;
+constexpr int kMaxShared = 8;
+constexpr int kTileRows = 128;     // weight rows per GEMM work unit (MMA M)
+constexpr int kTileK = 64;         // bf16 elements per 128-byte swizzled row
+constexpr int kRowPad = 16;        // expert segments are padded to this many rows (MMA N step)
+constexpr int kPermBlock = 256;    // tokens per block in the permute kernels
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
+
+// Byte offsets of every workspace region, plus the tiling chosen for a shape.
+struct Plan {
+  // shape
+  int T, d, E, k, f, S, fs;
+  // derived sizes
+  int Tp;          // T rounded up to kRowPad
+  int Rcap;        // routed row capacity: T*k + E*(kRowPad-1), rounded to kRowPad
+  int nb;          // permute blocks: ceil(T / kPermBlock)
+  int nmax_r;      // tokens per router work unit
+  int nmax1;       // rows per gate/up work unit (MMA N max)
+  int nmax2;       // rows per down work unit
+  int nwbE;        // 128-row blocks of E
+  int nwb1;        // 128-row blocks of f
+  int nwb1s;       // 128-row blocks of fs
+  int nwb2;        // 128-row blocks of d
+  int router_units;
+  int U1cap, U2cap;
+  int shared_units1, shared_units2;
+  // region offsets (bytes)
+  size_t err, nunits, logits, blkcnt, counts, roff, perm, roww, inv, units1, units2;
+  size_t Hr, Hs, Yr, Ys, xstage, ostage, istage, wstage;
+  size_t total;
+};
+
+// Fills `p` for `s`; returns MOE_OK or MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED.
+int make_plan(const moe_shape* s, Plan* p);
+
+// Per-device facts, looked up once per device.
+struct DeviceInfo {
+  int ok;          // 1 if sm_100 and attributes were read
+  int sms;
+  int max_smem_optin;
+};
+int device_info(DeviceInfo* info);
+
+// ---- kernel launchers (each returns MOE_OK or MOE_ERR_CUDA) ----
+enum GemmMode { kModeRouter = 0, kModeGateUp = 1, kModeDown = 2 };
+
+struct GemmParams {
+  CUtensorMap mapA[4];      // A operands: [0],[1] routed (gate, up | down | router); [2],[3] shared
+  CUtensorMap mapB[2];      // B sources: [0] routed / all tokens, [1] shared (down only)
+  const int4* units;        // work list (gate/up and down)
+  const int* num_units_dev; // its length, on the device
+  int num_units_host;       // router: number of units
+  const int* perm;          // gate/up: token of each routed row
+  const float* roww;        // down: combine weight of each routed row
+  void* out_r;              // router: logits f32 [T,E]; gate/up: H_r; down: Y_r
+  void* out_s;              // gate/up: H_s; down: Y_s
+  uint32_t* err;
+  int T, Tp, E, d, f, fs;
+  int nmax, stages, nbuf, router_nwb;
+  uint64_t timeout_ns;
+};
+
+int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st);
+size_t gemm_smem_bytes(int mode, int nmax, int* stages);
+
+int launch_topk(const float* logits, const float* bias, int T, int E, int k, int score_fn,
+                int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w,
+                cudaStream_t st);
+
+int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, char* ws,
+                   cudaStream_t st);
+
+int launch_combine(const Plan& p, void* out, const char* ws, cudaStream_t st);
+
+int launch_wait_timeout(uint32_t* err, uint64_t timeout_ns, cudaStream_t st);
+
+}  // namespace moe

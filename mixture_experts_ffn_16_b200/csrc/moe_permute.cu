@@ -1,0 +1,258 @@
+// moe_permute.cu - token -> expert dispatch (step a3), entirely on the device.
+//
+//   count   : per block of 256 tokens, a bit mask per (warp, expert) of the
+//             lanes whose token picked the expert; popcounts give the block's
+//             per-expert histogram.
+//   scan    : one block: per expert, exclusive prefix over blocks (-> each
+//             block's offset inside the expert's segment) and the expert's
+//             count; then exclusive scans over experts of the padded segment
+//             sizes and of the GEMM work-unit counts; writes the work lists
+//             and fills the padding rows.
+//   scatter : recomputes the masks; a (token, slot) pair's row is
+//             segment start + block offset + popcount of the lower lanes of
+//             the lower warps and of its own warp: rows inside an expert are in
+//             ascending token order, so the layout is deterministic.
+//
+// Row space: expert e owns rows [roff[e], roff[e] + pad16(count[e])); padding
+// rows point at token 0 with weight 0.  Work units are int4
+// {group, 128-row weight block, first row, rows (multiple of 16)}; shared
+// experts are groups E..E+S-1 over rows 0..pad16(T) of their own row space and
+// come first in each list.
+#include "moe_internal.h"
+#include "moe_ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kWarps = kPermBlock / 32;
+constexpr int kScanThreads = 1024;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Fills masks[w*E + e] for this block; flags invalid routing.
+__device__ void build_masks(const int32_t* __restrict__ topk_idx, int T, int E, int k,
+                            uint32_t* masks, uint32_t* err) {
+  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) masks[i] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kPermBlock + threadIdx.x;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (t < T) {
+    bool bad = false;
+    for (int j = 0; j < k; ++j) {
+      const int e = topk_idx[static_cast<size_t>(t) * k + j];
+      if (e < 0 || e >= E) {
+        bad = true;
+        continue;
+      }
+      const uint32_t old = atomicOr(&masks[w * E + e], 1u << lane);
+      if (old & (1u << lane)) bad = true;   // the same expert twice in one token
+    }
+    if (bad) atomicOr(err, kDevErrBadRouting);
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kPermBlock)
+permute_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
+                     int32_t* __restrict__ blkcnt, uint32_t* err) {
+  extern __shared__ uint32_t masks[];
+  build_masks(topk_idx, T, E, k, masks, err);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) c += __popc(masks[w * E + e]);
+    blkcnt[static_cast<size_t>(blockIdx.x) * E + e] = c;
+  }
+}
+
+// Exclusive block-wide scan of one int per thread (kScanThreads threads).
+__device__ int block_exclusive_scan(int v, int* sh, int* total) {
+  const int tid = threadIdx.x;
+  sh[tid] = v;
+  __syncthreads();
+  for (int off = 1; off < kScanThreads; off <<= 1) {
+    const int add = tid >= off ? sh[tid - off] : 0;
+    __syncthreads();
+    sh[tid] += add;
+    __syncthreads();
+  }
+  const int incl = sh[tid];
+  *total = sh[kScanThreads - 1];
+  __syncthreads();
+  return incl - v;
+}
+
+struct ScanArgs {
+  int32_t* blkcnt;   // [nb, E] in: counts, out: exclusive offsets over blocks
+  int32_t* counts;   // [E]
+  int32_t* roff;     // [E+1]
+  int32_t* perm;     // [Rcap]
+  float* roww;       // [Rcap]
+  int4* units1;
+  int4* units2;
+  int32_t* nunits;   // [4]: gate/up units, down units, padded routed rows, 0
+  int nb, E, T, Tp;
+  int nmax1, nmax2, nwb1, nwb1s, nwb2, S;
+  int shared_units1, shared_units2;
+};
+
+__global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) {
+  __shared__ int sh[kScanThreads];
+  // Experts per thread: E <= 2048 -> at most 2.
+  constexpr int kPer = (kMaxE + kScanThreads - 1) / kScanThreads;
+  int cnt[kPer], pad[kPer], u1[kPer], u2[kPer];
+  int sp = 0, s1 = 0, s2 = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = threadIdx.x * kPer + i;
+    int c = 0;
+    if (e < a.E) {
+      for (int b = 0; b < a.nb; ++b) {
+        int32_t* p = a.blkcnt + static_cast<size_t>(b) * a.E + e;
+        const int v = *p;
+        *p = c;
+        c += v;
+      }
+      a.counts[e] = c;
+    }
+    cnt[i] = c;
+    pad[i] = (c + kRowPad - 1) / kRowPad * kRowPad;
+    u1[i] = (pad[i] + a.nmax1 - 1) / a.nmax1 * a.nwb1;
+    u2[i] = (pad[i] + a.nmax2 - 1) / a.nmax2 * a.nwb2;
+    sp += pad[i];
+    s1 += u1[i];
+    s2 += u2[i];
+  }
+  int tot_rows, tot1, tot2;
+  int ro = block_exclusive_scan(sp, sh, &tot_rows);
+  int o1 = a.shared_units1 + block_exclusive_scan(s1, sh, &tot1);
+  int o2 = a.shared_units2 + block_exclusive_scan(s2, sh, &tot2);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = threadIdx.x * kPer + i;
+    if (e < a.E) {
+      a.roff[e] = ro;
+      // padding rows of this expert's segment
+      for (int r = cnt[i]; r < pad[i]; ++r) {
+        a.perm[ro + r] = 0;
+        a.roww[ro + r] = 0.0f;
+      }
+      // gate/up units: (e, wb, chunk), chunks inner so that consecutive units share a weight tile
+      const int nch1 = (pad[i] + a.nmax1 - 1) / a.nmax1;
+      for (int wb = 0; wb < a.nwb1; ++wb)
+        for (int c = 0; c < nch1; ++c)
+          a.units1[o1 + wb * nch1 + c] = make_int4(e, wb, ro + c * a.nmax1, min(a.nmax1, pad[i] - c * a.nmax1));
+      const int nch2 = (pad[i] + a.nmax2 - 1) / a.nmax2;
+      for (int wb = 0; wb < a.nwb2; ++wb)
+        for (int c = 0; c < nch2; ++c)
+          a.units2[o2 + wb * nch2 + c] = make_int4(e, wb, ro + c * a.nmax2, min(a.nmax2, pad[i] - c * a.nmax2));
+    }
+    ro += pad[i];
+    o1 += u1[i];
+    o2 += u2[i];
+  }
+  // Shared-expert units (first in each list).
+  const int nch1s = (a.Tp + a.nmax1 - 1) / a.nmax1;
+  const int nch2s = (a.Tp + a.nmax2 - 1) / a.nmax2;
+  for (int i = threadIdx.x; i < a.shared_units1; i += blockDim.x) {
+    const int c = i % nch1s, rest = i / nch1s;
+    const int wb = rest % a.nwb1s, s = rest / a.nwb1s;
+    a.units1[i] = make_int4(a.E + s, wb, c * a.nmax1, min(a.nmax1, a.Tp - c * a.nmax1));
+  }
+  for (int i = threadIdx.x; i < a.shared_units2; i += blockDim.x) {
+    const int c = i % nch2s, rest = i / nch2s;
+    const int wb = rest % a.nwb2, s = rest / a.nwb2;
+    a.units2[i] = make_int4(a.E + s, wb, c * a.nmax2, min(a.nmax2, a.Tp - c * a.nmax2));
+  }
+  if (threadIdx.x == 0) {
+    a.roff[a.E] = tot_rows;
+    a.nunits[0] = a.shared_units1 + tot1;
+    a.nunits[1] = a.shared_units2 + tot2;
+    a.nunits[2] = tot_rows;
+    a.nunits[3] = 0;
+  }
+}
+
+__global__ void __launch_bounds__(kPermBlock)
+permute_scatter_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w, int T,
+                       int E, int k, const int32_t* __restrict__ blkoff, const int32_t* __restrict__ roff,
+                       int32_t* __restrict__ perm, float* __restrict__ roww, int32_t* __restrict__ inv,
+                       uint32_t* err) {
+  extern __shared__ uint32_t masks[];
+  build_masks(topk_idx, T, E, k, masks, err);
+  const int t = blockIdx.x * kPermBlock + threadIdx.x;
+  if (t >= T) return;
+  const int w = threadIdx.x >> 5;
+  const uint32_t lt = lanemask_lt();
+  for (int j = 0; j < k; ++j) {
+    const size_t tj = static_cast<size_t>(t) * k + j;
+    const int e = topk_idx[tj];
+    if (e < 0 || e >= E) {
+      inv[tj] = roff[0];   // invalid routing was flagged; keep the index in range
+      continue;
+    }
+    int rank = __popc(masks[w * E + e] & lt);
+    for (int v = 0; v < w; ++v) rank += __popc(masks[v * E + e]);
+    const int row = roff[e] + blkoff[static_cast<size_t>(blockIdx.x) * E + e] + rank;
+    perm[row] = t;
+    roww[row] = topk_w[tj];
+    inv[tj] = row;
+  }
+}
+
+}  // namespace
+
+int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, char* ws,
+                   cudaStream_t st) {
+  int32_t* blkcnt = reinterpret_cast<int32_t*>(ws + p.blkcnt);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws + p.err);
+  const size_t msmem = static_cast<size_t>(kWarps) * p.E * sizeof(uint32_t);
+  static int configured[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  if (!configured[dev]) {
+    const int mx = kWarps * kMaxE * static_cast<int>(sizeof(uint32_t));
+    if (cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess ||
+        cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured[dev] = 1;
+  }
+  permute_count_kernel<<<p.nb, kPermBlock, msmem, st>>>(topk_idx, p.T, p.E, p.k, blkcnt, err);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+
+  ScanArgs a;
+  a.blkcnt = blkcnt;
+  a.counts = reinterpret_cast<int32_t*>(ws + p.counts);
+  a.roff = reinterpret_cast<int32_t*>(ws + p.roff);
+  a.perm = reinterpret_cast<int32_t*>(ws + p.perm);
+  a.roww = reinterpret_cast<float*>(ws + p.roww);
+  a.units1 = reinterpret_cast<int4*>(ws + p.units1);
+  a.units2 = reinterpret_cast<int4*>(ws + p.units2);
+  a.nunits = reinterpret_cast<int32_t*>(ws + p.nunits);
+  a.nb = p.nb;
+  a.E = p.E;
+  a.T = p.T;
+  a.Tp = p.Tp;
+  a.nmax1 = p.nmax1;
+  a.nmax2 = p.nmax2;
+  a.nwb1 = p.nwb1;
+  a.nwb1s = p.nwb1s;
+  a.nwb2 = p.nwb2;
+  a.S = p.S;
+  a.shared_units1 = p.shared_units1;
+  a.shared_units2 = p.shared_units2;
+  permute_scan_kernel<<<1, kScanThreads, 0, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+
+  permute_scatter_kernel<<<p.nb, kPermBlock, msmem, st>>>(
+      topk_idx, topk_w, p.T, p.E, p.k, blkcnt, a.roff, a.perm, a.roww,
+      reinterpret_cast<int32_t*>(ws + p.inv), err);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

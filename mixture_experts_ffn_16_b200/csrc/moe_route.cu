@@ -1,0 +1,148 @@
+// moe_route.cu - scoring, top-k selection and combine weights (step a2).
+//
+// One warp per token reads the token's fp32 logits (written by the router
+// GEMM), forms the scores and selection keys in registers, and picks the k
+// largest keys by k rounds of a warp-wide arg-max (ties go to the lower expert
+// index, matching a stable descending sort).
+//
+//   softmax       : key = logit (same order as the softmax probability);
+//                   w_j = exp(l_j - l_max) / (norm ? sum over picks : sum over all E)
+//   sigmoid       : s = 1/(1+exp(-l)),            key = s + bias
+//   sqrt-softplus : s = sqrt(max(l,0) + log1p(exp(-|l|))), key = s + bias
+//                   w_j = s_j (/ sum over picks if norm)
+//   then w_j *= route_scale.
+// The bias only orders the experts; the weights come from the unbiased scores.
+#include <cfloat>
+#include <cmath>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+
+__device__ __forceinline__ float score_of(float l, int fn) {
+  if (fn == MOE_SCORE_SIGMOID) return 1.0f / (1.0f + expf(-l));
+  // MOE_SCORE_SQRT_SOFTPLUS
+  return sqrtf(fmaxf(l, 0.0f) + log1pf(expf(-fabsf(l))));
+}
+
+// (key, idx) order: larger key first, then lower index.
+__device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
+  return (ka > kb) || (ka == kb && ia < ib);
+}
+
+template <int NPL>   // keys per lane: E <= 32 * NPL
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
+            int score_fn, int norm_topk, float route_scale, int32_t* __restrict__ topk_idx,
+            float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* row = logits + static_cast<size_t>(t) * E;
+  const bool use_bias = (bias != nullptr) && (score_fn != MOE_SCORE_SOFTMAX);
+
+  float key[NPL];
+  float lmax = -FLT_MAX;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    float kv = -INFINITY;
+    if (e < E) {
+      const float l = row[e];
+      lmax = fmaxf(lmax, l);
+      kv = (score_fn == MOE_SCORE_SOFTMAX) ? l : score_of(l, score_fn) + (use_bias ? bias[e] : 0.0f);
+    }
+    key[i] = kv;
+  }
+
+  // Softmax without renormalisation needs the full denominator.
+  float zsum = 0.0f;
+  if (score_fn == MOE_SCORE_SOFTMAX) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    if (!norm_topk) {
+#pragma unroll
+      for (int i = 0; i < NPL; ++i)
+        if (lane + 32 * i < E) zsum += expf(key[i] - lmax);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) zsum += __shfl_xor_sync(0xffffffffu, zsum, o);
+    }
+  }
+
+  int my_idx = -1;    // lane j keeps the j-th pick
+  for (int j = 0; j < k; ++j) {
+    float bk = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && better(key[i], e, bk, bi)) {
+        bk = key[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (better(ok, oi, bk, bi)) {
+        bk = ok;
+        bi = oi;
+      }
+    }
+    // Remove the winner (its owner lane), record it in lane j.
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (lane + 32 * i == bi) key[i] = -INFINITY;
+    if (lane == j) my_idx = bi;
+  }
+  // A removed key is -inf; a real -inf key could then be picked twice only if
+  // fewer than k experts have finite keys, which finite inputs never produce.
+
+  float s = 0.0f;
+  if (lane < k) {
+    const float l = row[my_idx];
+    s = (score_fn == MOE_SCORE_SOFTMAX) ? expf(l - lmax) : score_of(l, score_fn);
+  }
+  float denom;
+  if (norm_topk) {
+    denom = s;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
+    denom = fmaxf(denom, FLT_MIN);
+  } else {
+    denom = (score_fn == MOE_SCORE_SOFTMAX) ? zsum : 1.0f;
+  }
+  if (lane < k) {
+    topk_idx[static_cast<size_t>(t) * k + lane] = my_idx;
+    topk_w[static_cast<size_t>(t) * k + lane] = (s / denom) * route_scale;
+  }
+}
+
+template <int NPL>
+int launch_npl(const float* logits, const float* bias, int T, int E, int k, int fn, int norm,
+               float scale, int32_t* idx, float* w, cudaStream_t st) {
+  const int grid = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  topk_kernel<NPL><<<grid, kWarpsPerBlock * 32, 0, st>>>(logits, bias, T, E, k, fn, norm, scale, idx, w);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_topk(const float* logits, const float* bias, int T, int E, int k, int score_fn,
+                int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w,
+                cudaStream_t st) {
+  if (E <= 32) return launch_npl<1>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
+  if (E <= 64) return launch_npl<2>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
+  if (E <= 128) return launch_npl<4>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
+  if (E <= 256) return launch_npl<8>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
+  if (E <= 512) return launch_npl<16>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
+  if (E <= 1024) return launch_npl<32>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
+  return launch_npl<64>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,64 @@
+"""Algorithmic cost of the MoE block and of each of its kernels.
+
+Counts only what the method must do, not what an implementation moves:
+  FLOPs  2*M*N*K per GEMM: router (T x E x d), gate and up (T*k rows and S*T
+         shared rows, each 2 x f x d), down (same rows, d x f).
+  bytes  every weight matrix a kernel needs read once (routed experts only if
+         some token picked them), activations read once and results written
+         once, in their stored dtype.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def measured_peaks():
+    """Peaks measured on this machine's B200s (generated file), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def kernel_costs(cfg, touched=None):
+    """Per-step algorithmic (flops, bytes) of each step of the block.
+
+    touched: number of routed experts with at least one token (default: all E).
+    """
+    T, d, E, k, f, S, fs = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.S, cfg.fs
+    ne = E if touched is None else int(touched)
+    R = T * k
+    c = {}
+    # a1+a2: router GEMM (x, W_router in; fp32 logits out) + top-k (logits in, idx/w out)
+    c["route"] = (2.0 * T * E * d, 2.0 * (T * d + E * d) + 4.0 * T * E * 2 + 8.0 * T * k)
+    # a3: permute: read idx/w twice, write perm/row_w/inv
+    c["permute"] = (0.0, 8.0 * R * 2 + 12.0 * R)
+    # a4 + a6 gate/up: weights of touched experts and shared, x, H out
+    c["gate_up"] = (2.0 * (R * 2 * f * d + S * T * 2 * fs * d),
+                    2.0 * (ne * 2 * f * d + S * 2 * fs * d + T * d + R * f + S * T * fs))
+    # a5 + a6 down: W_down, H in, Y out
+    c["down"] = (2.0 * (R * d * f + S * T * d * fs),
+                 2.0 * (ne * d * f + S * d * fs + R * f + S * T * fs + R * d + S * T * d))
+    # a7 combine: Y rows in, out written
+    c["combine"] = (float((R + S * T) * d), 2.0 * ((R + S * T) * d + T * d) + 4.0 * R)
+    return c
+
+
+def block_cost(cfg, touched=None):
+    """Whole-block algorithmic (flops, bytes): the minimum any implementation
+    needs (weights of touched experts once, x in, out and routing out)."""
+    T, d, E, k, f, S, fs = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.S, cfg.fs
+    ne = E if touched is None else int(touched)
+    flops = 2.0 * T * E * d + 2.0 * T * k * 3 * f * d + 2.0 * T * S * 3 * fs * d
+    bytes_ = 2.0 * (ne * 3 * f * d + S * 3 * fs * d + E * d + 2 * T * d) + 8.0 * T * k
+    return flops, bytes_

@@ -54,7 +54,7 @@ def _load():
             i = ctypes.c_int
             lib.oracle_moe_forward.restype = i
             lib.oracle_moe_forward.argtypes = (
-                [i] * 7 + [P] * 3 + [P] * 6 + [i, i, ctypes.c_double] + [P, i, P, i] + [P] * 6 + [i])
+                [i] * 7 + [P] * 3 + [P] * 6 + [i, i, ctypes.c_double] + [P, i, P, i] + [P] * 8 + [i])
             _lib = lib
     return _lib
 
@@ -89,9 +89,10 @@ def forward(x, W_router, W_gate=None, W_up=None, W_down=None,
     order); ``forced_idx`` [n,k] replaces the router's choice of experts (the
     weights are then the scores of the forced experts, renormalised the same
     way).  Returns a dict of float64/int32 numpy arrays: ``out`` [n,d],
-    ``topk_idx`` [n,k], ``topk_w`` [n,k], ``sel_keys`` [n,k+1] (selection keys
-    of the first k+1 experts in selection order), and with ``want_logits``
-    also ``logits`` and ``scores`` [n,E].
+    ``topk_idx`` [n,k], ``topk_w`` [n,k], ``sel_keys`` / ``sel_order`` [n,k+1]
+    (selection keys and experts of the first k+1 in selection order; -inf / -1
+    past E), and with ``want_logits`` also ``logits``, ``scores`` and the
+    selection ``keys`` [n,E].
     """
     lib = _load()
     T, d = x.shape
@@ -129,8 +130,10 @@ def forward(x, W_router, W_gate=None, W_up=None, W_down=None,
     topk_idx = np.zeros((n, k), np.int32)
     topk_w = np.zeros((n, k), np.float64)
     sel_keys = np.zeros((n, k + 1), np.float64)
+    sel_order = np.zeros((n, k + 1), np.int32)
     logits = np.zeros((n, E), np.float64) if want_logits else None
     scores = np.zeros((n, E), np.float64) if want_logits else None
+    keys = np.zeros((n, E), np.float64) if want_logits else None
     if n_threads is None:
         n_threads = os.cpu_count() or 1
     st = lib.oracle_moe_forward(
@@ -141,14 +144,16 @@ def forward(x, W_router, W_gate=None, W_up=None, W_down=None,
         SCORE_FNS[score_fn] if isinstance(score_fn, str) else int(score_fn),
         int(bool(norm_topk)), float(route_scale),
         _ptr(tok), n, _ptr(forced), int(bool(route_only)),
-        _ptr(out), _ptr(topk_idx), _ptr(topk_w), _ptr(sel_keys),
-        _ptr(logits), _ptr(scores), int(n_threads))
+        _ptr(out), _ptr(topk_idx), _ptr(topk_w), _ptr(sel_keys), _ptr(sel_order),
+        _ptr(logits), _ptr(scores), _ptr(keys), int(n_threads))
     if st != 0:
         raise ValueError(f"oracle_moe_forward failed with status {st}")
-    res = {"out": out, "topk_idx": topk_idx, "topk_w": topk_w, "sel_keys": sel_keys}
+    res = {"out": out, "topk_idx": topk_idx, "topk_w": topk_w, "sel_keys": sel_keys,
+           "sel_order": sel_order}
     if want_logits:
         res["logits"] = logits
         res["scores"] = scores
+        res["keys"] = keys
     return res
 
 

@@ -151,8 +151,10 @@ typedef struct {
     int32_t *topk_idx;       /* [n_tokens,k] or NULL */
     double *topk_w;          /* [n_tokens,k] or NULL */
     double *sel_keys;        /* [n_tokens,k+1] selection keys in picked order (k+1-th = -inf if k == E) */
+    int32_t *sel_order;      /* [n_tokens,k+1] the experts of those keys (k+1-th = -1 if k == E) */
     double *logits_out;      /* [n_tokens,E] or NULL */
     double *scores_out;      /* [n_tokens,E] or NULL */
+    double *keys_out;        /* [n_tokens,E] selection keys, or NULL */
     int next;                /* work counter */
     pthread_mutex_t mu;
     int status;
@@ -184,10 +186,16 @@ static int oracle_token(oracle_job *J, int n, double *logit, double *s, keyed *k
         kv[e].key = s[e] + (use_bias ? (double)J->bias[e] : 0.0);
         kv[e].idx = e;
     }
+    if (J->keys_out)
+        for (int e = 0; e < E; ++e) J->keys_out[(size_t)n * E + e] = kv[e].key;
     qsort(kv, (size_t)E, sizeof(keyed), keyed_cmp);
     if (J->sel_keys) {
         double *sk = J->sel_keys + (size_t)n * (k + 1);
         for (int j = 0; j <= k; ++j) sk[j] = (j < E) ? kv[j].key : -INFINITY;
+    }
+    if (J->sel_order) {
+        int32_t *so = J->sel_order + (size_t)n * (k + 1);
+        for (int j = 0; j <= k; ++j) so[j] = (j < E) ? kv[j].idx : -1;
     }
 
     int sel[64];
@@ -266,7 +274,8 @@ int oracle_moe_forward(int T, int d, int E, int k, int f, int S, int fs,
                        const int32_t *tokens, int n_tokens, const int32_t *forced,
                        int route_only,
                        double *out, int32_t *topk_idx, double *topk_w, double *sel_keys,
-                       double *logits_out, double *scores_out, int n_threads)
+                       int32_t *sel_order, double *logits_out, double *scores_out, double *keys_out,
+                       int n_threads)
 {
     if (T < 1 || d < 1 || E < 1 || k < 1 || k > E || k > 64 || n_tokens < 0) return -1;
     if (score_fn < 0 || score_fn > 2 || !x || !Wr) return -1;
@@ -283,7 +292,8 @@ int oracle_moe_forward(int T, int d, int E, int k, int f, int S, int fs,
     J.score_fn = score_fn; J.norm_topk = norm_topk; J.route_scale = route_scale;
     J.tokens = tokens; J.n_tokens = n_tokens; J.forced = forced; J.route_only = route_only;
     J.out = out; J.topk_idx = topk_idx; J.topk_w = topk_w; J.sel_keys = sel_keys;
-    J.logits_out = logits_out; J.scores_out = scores_out;
+    J.sel_order = sel_order;
+    J.logits_out = logits_out; J.scores_out = scores_out; J.keys_out = keys_out;
     pthread_mutex_init(&J.mu, NULL);
 
     pthread_t th[512];

@@ -1,0 +1,123 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+function include/moe.h declares, and its host-side logic (workspace sizing,
+region layout, argument checks) behaves; nothing here launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_ffn_16_b200 import api, build
+from mixture_experts_ffn_16_b200.inputs import CONFIGS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.load()
+
+
+def declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fn in sorted(os.listdir(inc)):
+        if fn.endswith(".h"):
+            with open(os.path.join(inc, fn)) as fh:
+                src = fh.read()
+            names += re.findall(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", src)
+    return names
+
+
+def test_library_exports_every_declared_function(lib):
+    names = declared_functions()
+    assert len(names) >= 13
+    assert sorted(names) == sorted(api.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.moe_version() >= 100
+    for code in (0, -1, -2, -3, -4, -5):
+        assert lib.moe_status_string(code)
+    assert b"unknown" in lib.moe_status_string(42)
+
+
+@pytest.mark.parametrize("name", list(CONFIGS))
+def test_workspace_sizes_of_workloads(lib, name):
+    c = CONFIGS[name]
+    s = api.shape_of(c)
+    n = api.moe_workspace_bytes(s)
+    assert n > 0
+    # must at least hold the routed hidden and output rows (T*k of each) and the logits
+    assert n >= c.T * c.k * (c.f + c.d) * 2 + c.T * c.E * 4
+    # regions are disjoint, 256-byte aligned and inside the workspace
+    spans = []
+    for r in api.WS_REGIONS:
+        off, nb = api.moe_workspace_region(s, r)
+        assert off % 256 == 0 and off + nb <= n
+        spans.append((off, off + nb))
+    spans.sort()
+    for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+        assert a1 <= b0 or a0 == a1 or b0 == b1
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(T=0), api.MOE_ERR_INVALID_ARG), (dict(k=0), api.MOE_ERR_INVALID_ARG),
+    (dict(k=9, E=8), api.MOE_ERR_INVALID_ARG), (dict(E=0), api.MOE_ERR_INVALID_ARG),
+    (dict(d_model=100), api.MOE_ERR_UNSUPPORTED), (dict(d_ff=96), api.MOE_ERR_UNSUPPORTED),
+    (dict(n_shared=1, d_ff_shared=80), api.MOE_ERR_UNSUPPORTED), (dict(E=4096), api.MOE_ERR_UNSUPPORTED),
+    (dict(k=33, E=64), api.MOE_ERR_UNSUPPORTED), (dict(n_shared=9, d_ff_shared=64), api.MOE_ERR_UNSUPPORTED),
+])
+def test_invalid_shapes(lib, bad, code):
+    base = dict(T=16, d_model=128, E=8, k=2, d_ff=128, n_shared=1, d_ff_shared=128)
+    base.update(bad)
+    s = api.make_shape(**base)
+    assert api.moe_workspace_bytes(s) == 0
+    st = lib.moe_forward(ctypes.byref(s), *([ctypes.c_void_p(256)] * 9), 0, 1, 1.0,
+                         *([ctypes.c_void_p(256)] * 4), 1 << 30, None)
+    assert st == code
+
+
+def test_argument_checks_before_any_device_work(lib):
+    s = api.make_shape(16, 128, 8, 2, 128, 1, 128)
+    n = api.moe_workspace_bytes(s)
+    P = ctypes.c_void_p
+    good = [P(4096)] * 9
+    # null x
+    st = lib.moe_forward(ctypes.byref(s), None, *good[1:], 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096),
+                         n, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    # bad score function / norm flag / non-finite scale
+    for sf, nt, sc in [(3, 1, 1.0), (0, 2, 1.0), (0, 1, float("inf"))]:
+        st = lib.moe_forward(ctypes.byref(s), *good, sf, nt, sc, P(4096), P(4096), P(4096), P(4096), n, None)
+        assert st == api.MOE_ERR_INVALID_ARG
+    # misaligned pointer
+    st = lib.moe_forward(ctypes.byref(s), P(4098), *good[1:], 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096),
+                         n, None)
+    assert st == api.MOE_ERR_UNSUPPORTED
+    # shared weights given with S == 0
+    s0 = api.make_shape(16, 128, 8, 2, 128, 0, 0)
+    st = lib.moe_forward(ctypes.byref(s0), *good, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096),
+                         api.moe_workspace_bytes(s0), None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    # workspace too small / misaligned
+    st = lib.moe_forward(ctypes.byref(s), *good, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096), n - 1, None)
+    assert st == api.MOE_ERR_WORKSPACE
+    st = lib.moe_forward(ctypes.byref(s), *good, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4128), n, None)
+    assert st == api.MOE_ERR_WORKSPACE
+
+
+def test_region_query_rejects_bad_region(lib):
+    s = api.make_shape(16, 128, 8, 2, 128, 1, 128)
+    off, nb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.moe_workspace_region(ctypes.byref(s), 99, ctypes.byref(off), ctypes.byref(nb)) == api.MOE_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(api, "_lib", None)
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        api.load()

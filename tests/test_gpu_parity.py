@@ -1,0 +1,126 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on a B200.
+
+Small and medium shapes are checked on every token; they span several weight
+tiles, several token runs per expert, ragged tails (T, f, fs not multiples of
+the tile) and the degenerate cases (T=1, E=1, k=E, no shared expert, empty
+experts, minimum widths, the largest E and k).  The five workloads are run at
+full size in the launch configuration the benchmark times and checked on a
+seeded sample of tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_ffn_16_b200 import api
+from mixture_experts_ffn_16_b200.inputs import CONFIGS, MoEConfig, make_inputs, oracle_args
+
+from parity_util import check_parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    api.load()
+
+
+def run_gpu(cfg, inp):
+    layer = api.MoELayer(cfg, inp)
+    out, idx, w = layer()
+    st = api.moe_device_status(layer.workspace)
+    assert st == api.MOE_OK, api.status_string(st)
+    return out.float().cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy(), layer
+
+
+def parity_case(oracle_mod, cfg, tokens=None):
+    _need_gpu()
+    inp = make_inputs(cfg, device="cuda")
+    out, idx, w, _ = run_gpu(cfg, inp)
+    host = oracle_args(inp)
+    if tokens is not None:
+        out, idx, w = out[tokens], idx[tokens], w[tokens]
+    rep = check_parity(oracle_mod, cfg, host, out, idx, w, tokens=tokens)
+    print(cfg.name, rep)
+    return rep, inp
+
+
+MEDIUM = [
+    MoEConfig("med_softmax_ragged", T=300, d=512, E=40, k=6, f=192, S=1, fs=320, seed=11),
+    MoEConfig("med_sigmoid_bias_s2_scaled", T=257, d=384, E=24, k=4, f=256, S=2, fs=128,
+              score_fn="sigmoid", bias_std=0.1, route_scale=2.5, seed=12),
+    MoEConfig("med_sqrt_softplus_unnorm", T=200, d=256, E=33, k=5, f=128, S=1, fs=192,
+              score_fn="sqrt_softplus", bias_std=0.1, norm_topk=False, seed=13),
+    MoEConfig("med_softmax_unnorm_noshared", T=129, d=320, E=17, k=3, f=64, S=0, fs=0,
+              norm_topk=False, seed=14),
+    MoEConfig("dense_E1_k1", T=70, d=192, E=1, k=1, f=320, S=1, fs=64, seed=15),
+    MoEConfig("k_equals_E", T=50, d=128, E=6, k=6, f=128, S=0, fs=0, score_fn="sigmoid",
+              bias_std=0.5, seed=16),
+    MoEConfig("single_token", T=1, d=256, E=16, k=4, f=128, S=1, fs=128, seed=17),
+    MoEConfig("minimum_widths", T=17, d=64, E=5, k=2, f=64, S=1, fs=64, seed=18),
+    MoEConfig("many_chunks_per_expert", T=2000, d=256, E=4, k=2, f=128, S=1, fs=128, seed=19),
+    MoEConfig("max_E_and_k", T=48, d=128, E=2048, k=32, f=64, S=1, fs=64, seed=20),
+    MoEConfig("E896_like_large", T=96, d=256, E=896, k=22, f=64, S=2, fs=128, seed=21),
+    MoEConfig("multi_tile_medium", T=1000, d=1024, E=64, k=8, f=256, S=1, fs=256,
+              score_fn="sigmoid", bias_std=0.1, seed=22),
+]
+
+
+def test_tiny_workload_every_token(oracle_mod):
+    rep, _ = parity_case(oracle_mod, CONFIGS["tiny"])
+    assert rep["tokens"] == 64
+
+
+@pytest.mark.parametrize("cfg", MEDIUM, ids=lambda c: c.name)
+def test_medium_shapes_every_token(oracle_mod, cfg):
+    parity_case(oracle_mod, cfg)
+
+
+def test_empty_and_overloaded_experts(oracle_mod):
+    """A selection bias that sends every token to the same experts: most
+    experts get no rows, two get all T rows (several token runs each)."""
+    _need_gpu()
+    cfg = MoEConfig("skewed_bias", T=700, d=256, E=32, k=2, f=128, S=1, fs=128,
+                    score_fn="sigmoid", bias_std=0.1, seed=23)
+    inp = make_inputs(cfg, device="cuda")
+    inp["expert_bias"][5] = 50.0
+    inp["expert_bias"][9] = 40.0
+    out, idx, w, layer = run_gpu(cfg, inp)
+    assert (np.sort(idx, 1) == [5, 9]).all()
+    counts = api.workspace_view(layer.workspace, layer.shape, "counts", torch.int32, (cfg.E,)).cpu().numpy()
+    assert counts[5] == cfg.T and counts[9] == cfg.T and counts.sum() == cfg.T * cfg.k
+    check_parity(oracle_mod, cfg, oracle_args(inp), out, idx, w)
+
+
+def _sample(T, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(T, size=min(n, T), replace=False)).astype(np.int32)
+
+
+@pytest.mark.parametrize("name,n_tok", [("prefill_softmax", 384), ("prefill_sigmoid", 128),
+                                        ("decode_sqrt_softplus", 64), ("large_imbalanced", 48)])
+def test_full_size_workloads_sampled(oracle_mod, name, n_tok):
+    cfg = CONFIGS[name]
+    _need_gpu()
+    inp = make_inputs(cfg, device="cuda")
+    out, idx, w, layer = run_gpu(cfg, inp)
+    # properties at any size: finite output, valid routing, weights sum to route_scale
+    assert np.isfinite(out).all()
+    assert ((idx >= 0) & (idx < cfg.E)).all()
+    assert all(len(set(r)) == cfg.k for r in idx[: min(cfg.T, 4096)].tolist())
+    if cfg.norm_topk:
+        np.testing.assert_allclose(w.sum(1), cfg.route_scale, rtol=1e-5)
+    counts = np.bincount(idx.ravel(), minlength=cfg.E)
+    dev_counts = api.workspace_view(layer.workspace, layer.shape, "counts", torch.int32,
+                                    (cfg.E,)).cpu().numpy()
+    assert np.array_equal(counts, dev_counts)
+    if cfg.skew:
+        nz = counts[counts > 0]
+        ratio = np.inf if (counts == 0).any() else counts.max() / counts.min()
+        print(name, "expert load max/min", ratio, "max", counts.max(), "min nonzero", nz.min(),
+              "empty", int((counts == 0).sum()))
+        assert ratio > 10
+    tokens = _sample(cfg.T, n_tok, seed=cfg.seed + 100)
+    host = oracle_args(inp)
+    rep = check_parity(oracle_mod, cfg, host, out[tokens], idx[tokens], w[tokens], tokens=tokens)
+    print(name, rep)

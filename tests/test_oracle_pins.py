@@ -156,6 +156,7 @@ def test_topk_brute_force(oracle_mod, E, k, score_fn, with_bias):
         key = s + (bias.astype(np.float64) if (bias is not None and score_fn != "softmax") else 0.0)
         order = sorted(range(E), key=lambda e: (-key[e], e))
         assert r["topk_idx"][t].tolist() == order[:k]
+        assert r["sel_order"][t][:min(k + 1, E)].tolist() == order[:k + 1]
         np.testing.assert_array_equal(r["sel_keys"][t][:min(k + 1, E)],
                                       [key[e] for e in order[:k + 1]])
 
@@ -360,3 +361,16 @@ def test_invalid_arguments_rejected(oracle_mod):
         oracle_mod.forward(**c, k=4)           # k > E
     with pytest.raises(ValueError):
         oracle_mod.forward(**c, k=1, tokens=[0, 9])   # token out of range
+
+
+def test_keys_are_scores_plus_bias_for_biased_routers(oracle_mod):
+    rng = np.random.default_rng(19)
+    c = rand_case(rng, 5, 16, 6, 8)
+    b = rng.normal(0, 0.3, 6).astype(np.float32)
+    for fn in ["softmax", "sigmoid", "sqrt_softplus"]:
+        r = oracle_mod.forward(c["x"], c["W_router"], expert_bias=b, k=2, score_fn=fn,
+                               route_only=True, want_logits=True)
+        ref = r["scores"] + (0.0 if fn == "softmax" else b.astype(np.float64))
+        assert np.array_equal(r["keys"], ref)
+        np.testing.assert_array_equal(np.take_along_axis(r["keys"], r["sel_order"][:, :3], 1),
+                                      r["sel_keys"][:, :3])
