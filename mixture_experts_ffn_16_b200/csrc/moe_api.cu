@@ -48,16 +48,18 @@ bool map_weights(CUtensorMap* m, const void* ptr, int K, int rows, int G) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row-gather source [rows, K] bf16: box of one row x 64 K, 128-byte swizzle.
-bool map_rows(CUtensorMap* m, const void* ptr, int K, int rows) {
+// Token-row source [rows, K] bf16, 128-byte swizzle.  box_rows = 1 for the
+// gather4 loads (one row high box), kRowPad for tiled loads of 16 rows.
+bool map_rows(CUtensorMap* m, const void* ptr, int K, int rows, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), 1};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            box_rows == 1 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -87,7 +89,7 @@ int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_
   if (cudaMemsetAsync(ws + p.err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
   GemmParams g;
   std::memset(&g, 0, sizeof g);
-  if (!map_weights(&g.mapA[0], W_router, p.d, p.E, 1) || !map_rows(&g.mapB[0], x, p.d, p.T))
+  if (!map_weights(&g.mapA[0], W_router, p.d, p.E, 1) || !map_rows(&g.mapB[0], x, p.d, p.T, kRowPad))
     return MOE_ERR_CUDA;
   g.mapA[1] = g.mapA[2] = g.mapA[3] = g.mapA[0];
   g.mapB[1] = g.mapB[0];
@@ -114,7 +116,7 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* 
   GemmParams g;
   std::memset(&g, 0, sizeof g);
   if (!map_weights(&g.mapA[0], Wg, p.d, p.f, p.E) || !map_weights(&g.mapA[1], Wu, p.d, p.f, p.E) ||
-      !map_rows(&g.mapB[0], x, p.d, p.T))
+      !map_rows(&g.mapB[0], x, p.d, p.T, 1))
     return MOE_ERR_CUDA;
   if (p.S > 0) {
     if (!map_weights(&g.mapA[2], Wsg, p.d, p.fs, p.S) || !map_weights(&g.mapA[3], Wsu, p.d, p.fs, p.S))
@@ -127,6 +129,7 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* 
   g.units = reinterpret_cast<const int4*>(ws + p.units1);
   g.num_units_dev = reinterpret_cast<const int*>(ws + p.nunits);
   g.perm = reinterpret_cast<const int*>(ws + p.perm);
+  g.x = x;
   g.out_r = ws + p.Hr;
   g.out_s = ws + p.Hs;
   g.err = reinterpret_cast<uint32_t*>(ws + p.err);
@@ -143,10 +146,10 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* 
 int run_down(const Plan& p, const DeviceInfo& di, const void* Wd, const void* Wsd, char* ws, cudaStream_t st) {
   GemmParams g;
   std::memset(&g, 0, sizeof g);
-  if (!map_weights(&g.mapA[0], Wd, p.f, p.d, p.E) || !map_rows(&g.mapB[0], ws + p.Hr, p.f, p.Rcap))
+  if (!map_weights(&g.mapA[0], Wd, p.f, p.d, p.E) || !map_rows(&g.mapB[0], ws + p.Hr, p.f, p.Rcap, kRowPad))
     return MOE_ERR_CUDA;
   if (p.S > 0) {
-    if (!map_weights(&g.mapA[2], Wsd, p.fs, p.d, p.S) || !map_rows(&g.mapB[1], ws + p.Hs, p.fs, p.S * p.Tp))
+    if (!map_weights(&g.mapA[2], Wsd, p.fs, p.d, p.S) || !map_rows(&g.mapB[1], ws + p.Hs, p.fs, p.S * p.Tp, kRowPad))
       return MOE_ERR_CUDA;
   } else {
     g.mapA[2] = g.mapA[0];

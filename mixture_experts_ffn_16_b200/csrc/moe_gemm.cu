@@ -33,7 +33,11 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kGatherWarps = 4;                      // gate/up: warps that gather token rows
+constexpr int kGatherThreads = 32 * kGatherWarps;
+__host__ __device__ constexpr int threads_of(int mode) {
+  return mode == kModeGateUp ? 192 + kGatherThreads : 192;
+}
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kATileBytes = kTileRows * 128;   // 128 weight rows x 64 bf16
 constexpr int kEpiStageBytes = 2048;                 // per epilogue warp
@@ -77,7 +81,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1) moe_gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr int NA = (MODE == kModeGateUp) ? 2 : 1;   // A operands (accumulators) per unit
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -99,7 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_gemm_kernel(const __grid_cons
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full + s, 1);
+      // gate/up: the weight-tile producer's arrival plus one per gathering thread
+      mbar_init(full + s, MODE == kModeGateUp ? 1 + kGatherThreads : 1);
       mbar_init(empty + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -140,58 +145,38 @@ __global__ void __launch_bounds__(kThreads, 1) moe_gemm_kernel(const __grid_cons
       const CUtensorMap* mA = &p.mapA[sh ? 2 : 0];
       const CUtensorMap* mB = &p.mapB[(MODE == kModeDown && sh) ? 1 : 0];
       const int a_c2 = (MODE == kModeRouter) ? 0 : (sh ? sidx : un.g);
-      // Source rows of this lane's gathers: quads q = lane and lane + 32.
-      int rows[2][4];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int i = 4 * (lane + 32 * j) + r;
-          int src = 0;
-          if (i < un.n) {
-            if (MODE == kModeRouter) {
-              src = min(un.row0 + i, p.T - 1);
-            } else if (MODE == kModeGateUp) {
-              src = sh ? min(un.row0 + i, p.T - 1) : __ldg(p.perm + un.row0 + i);
-            } else {
-              src = sh ? sidx * p.Tp + un.row0 + i : un.row0 + i;
-            }
+      // Router / down: the unit's rows are contiguous in the source; first row:
+      const int brow0 = (MODE == kModeDown && sh) ? sidx * p.Tp + un.row0 : un.row0;
+      // Gate/up token rows come from the gather warps, not from TMA.
+      const uint32_t tx_bytes =
+          NA * kATileBytes + (MODE == kModeGateUp ? 0u : static_cast<uint32_t>(un.n) * 128u);
+      int got = 1;
+      if (lane == 0) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
+            got = 0;
+            break;
           }
-          rows[j][r] = src;
-        }
-      }
-      const uint32_t tx_bytes = NA * kATileBytes + static_cast<uint32_t>(un.n) * 128u;
-      for (int kb = 0; kb < KB; ++kb) {
-        int got = 1;
-        if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) {
-          ok = false;
-          break;
-        }
-        const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
-        const uint32_t fb = smem_u32(&full[stage]);
-        if (lane == 0) {
+          const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+          const uint32_t fb = smem_u32(&full[stage]);
           mbar_arrive_expect_tx(&full[stage], tx_bytes);
 #pragma unroll
           for (int a = 0; a < NA; ++a)
             tma_load_3d(sbase + a * kATileBytes, mA + a, fb, kb * kTileK, un.wb * kTileRows, a_c2);
-        }
-        __syncwarp();
-        const uint32_t bbase = sbase + NA * kATileBytes;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int qd = lane + 32 * j;
-          if (4 * qd < un.n)
-            tma_gather4(bbase + qd * 512u, mB, fb, kb * kTileK, rows[j][0], rows[j][1], rows[j][2],
-                        rows[j][3]);
-        }
-        ++issued;
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
+          if (MODE != kModeGateUp) {
+            const uint32_t bbase = sbase + NA * kATileBytes;
+            for (int i = 0; i < (un.n >> 4); ++i)
+              tma_load_2d(bbase + i * 2048u, mB, fb, kb * kTileK, brow0 + 16 * i);
+          }
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) ok = false;
     }
     // Leave no copy in flight: the last min(S, issued) stages armed.
     if (lane == 0) {
@@ -226,6 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1) moe_gemm_kernel(const __grid_cons
             break;
           }
           tc_fence_after();
+          // Token rows written by cp.async (generic proxy) are read by the
+          // tensor cores (async proxy).
+          if (MODE == kModeGateUp) fence_proxy_async_smem();
           const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
           const uint64_t bdesc = sw128_kmajor_desc(sbase + NA * kATileBytes);
           uint64_t adesc[NA];
@@ -256,7 +244,55 @@ __global__ void __launch_bounds__(kThreads, 1) moe_gemm_kernel(const __grid_cons
       }
     }
     __syncwarp();
-  } else {
+  } else if (MODE == kModeGateUp && warp >= 6) {
+    // ------------------------------------------------------------ row gather
+    // Thread g copies 16-byte chunk (g & 7) of rows (g >> 3) + 16 i of the
+    // token tile, i < n / 16, into the 128-byte-swizzled slot: chunk c of row
+    // r lands at r * 128 + ((c ^ (r & 7)) * 16).
+    const int g = threadIdx.x - 192;
+    const int part = g & 7;
+    const int r0 = g >> 3;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      const Unit un = get_unit<MODE>(p, u);
+      const bool sh = un.g >= p.E;
+      const int nr = un.n >> 4;                    // rows of this thread
+      int tok[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = un.row0 + r0 + 16 * i;
+        // clamped: a row never reads outside x, even for an invalid routing
+        tok[i] = (i < nr) ? min(max(sh ? r : __ldg(p.perm + r), 0), p.T - 1) : 0;
+      }
+      const int KB = p.d / kTileK;
+      for (int kb = 0; kb < KB; ++kb) {
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          ok = false;
+          break;
+        }
+        const uint32_t bbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + NA * kATileBytes;
+        const __nv_bfloat16* src0 = reinterpret_cast<const __nv_bfloat16*>(p.x) + kb * kTileK + part * 8;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (i < nr) {
+            const int r = r0 + 16 * i;
+            cp_async_16(bbase + r * 128 + ((part ^ (r & 7)) << 4), src0 + static_cast<size_t>(tok[i]) * p.d);
+          }
+        }
+        cp_async_mbar_arrive_noinc(&full[stage]);
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    cp_async_wait_all();
+  } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                       // TMEM lane quarter this warp may read
     uint8_t* stg = epi + (warp - 2) * kEpiStageBytes;
@@ -381,7 +417,7 @@ static int launch_mode(const GemmParams& prm, int grid, size_t smem, cudaStream_
       return MOE_ERR_CUDA;
     configured[dev] = static_cast<int>(smem);
   }
-  moe_gemm_kernel<MODE><<<grid, kThreads, smem, st>>>(prm);
+  moe_gemm_kernel<MODE><<<grid, threads_of(MODE), smem, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -67,6 +67,7 @@ struct GemmParams {
   int num_units_host;       // router: number of units
   const int* perm;          // gate/up: token of each routed row
   const float* roww;        // down: combine weight of each routed row
+  const void* x;            // gate/up: the tokens [T,d] bf16 (row gather source)
   void* out_r;              // router: logits f32 [T,E]; gate/up: H_r; down: Y_r
   void* out_s;              // gate/up: H_s; down: Y_s
   uint32_t* err;

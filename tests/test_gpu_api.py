@@ -86,6 +86,7 @@ def test_permute_matches_brute_force_counting_sort(T, E, k):
         pytest.skip("no CUDA device")
     shape = api.make_shape(T, 128, E, k, 128, 1, 128)
     ws = api.alloc_workspace(shape)
+    ws.zero_()       # the error word is cleared by moe_route, which this test skips
     idx, w = _synthetic_routing(T, E, k, seed=T + E + k)
     api.moe_permute(shape, idx.cuda(), w.cuda(), ws)
     torch.cuda.synchronize()
@@ -121,6 +122,7 @@ def test_invalid_routing_is_reported_not_faulted():
     T, E, k = 40, 8, 2
     shape = api.make_shape(T, 128, E, k, 128, 0, 0)
     ws = api.alloc_workspace(shape)
+    ws.zero_()
     idx = torch.zeros((T, k), dtype=torch.int32)
     idx[:, 1] = 1
     idx[3, 1] = 0          # repeated expert
