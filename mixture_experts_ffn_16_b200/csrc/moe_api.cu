@@ -103,7 +103,7 @@ int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_
   int stages = 0;
   const size_t smem = gemm_smem_bytes(kModeRouter, p.nmax_r, &stages);
   g.stages = stages;
-  g.nbuf = (p.nmax_r <= 256) ? 2 : 1;
+  g.nbuf = 512 / p.nmax_r < 8 ? 512 / p.nmax_r : 8;   // partial-logit buffers drained in turn
   const int grid = p.router_units < di.sms ? p.router_units : di.sms;
   int rc = launch_gemm(kModeRouter, g, grid, smem, st);
   if (rc != MOE_OK) return rc;
@@ -233,10 +233,11 @@ int make_plan(const moe_shape* s, Plan* p) {
   const double rows_per_expert = static_cast<double>(T) * k / E;
   q.nmax1 = pick_nmax(rows_per_expert);
   q.nmax2 = q.nmax1;
-  // Router: the widest token run that still gives every SM of a B200 a unit.
+  // Router: runs of up to 64 tokens (their fp32 logit sums live in registers);
+  // narrower runs only when that leaves most SMs of a B200 idle.
   q.nmax_r = 16;
-  for (int n = 256; n >= 16; n >>= 1) {
-    if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, n) >= 148) {
+  for (int n = 64; n >= 16; n >>= 1) {
+    if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, n) >= 74) {
       q.nmax_r = n;
       break;
     }

@@ -43,7 +43,10 @@ constexpr uint32_t kATileBytes = kTileRows * 128;   // 128 weight rows x 64 bf16
 constexpr int kEpiStageBytes = 2048;                 // per epilogue warp
 constexpr int kMaxStages = 8;
 constexpr int kSmemAlign = 1024;
-constexpr int kSmemTail = 256;                       // barriers, TMEM slot, abort flag
+constexpr int kSmemTail = 512;                       // barriers, TMEM slot, abort flag
+constexpr int kMaxTmemBufs = 8;                      // accumulator buffers (router: 8 x 64 columns)
+constexpr int kRouterDrainKB = 2;                    // router: k-blocks accumulated in TMEM per drain
+constexpr int kRouterMaxN = 64;                      // router: tokens per unit (fp32 sums in registers)
 
 struct Unit {
   int g, wb, row0, n;
@@ -93,8 +96,8 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
   uint64_t* full = reinterpret_cast<uint64_t*>(epi + 4 * kEpiStageBytes);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* tempty = tfull + kMaxTmemBufs;
+  uint64_t* drain = tempty + kMaxTmemBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
       mbar_init(full + s, MODE == kModeGateUp ? 1 + kGatherThreads : 1);
       mbar_init(empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kMaxTmemBufs; ++b) {
       mbar_init(tfull + b, 1);
       mbar_init(tempty + b, 4);
     }
@@ -194,48 +197,95 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
       uint32_t ucount = 0;
       bool any = false;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const Unit un = get_unit<MODE>(p, u);
-        const bool sh = (MODE != kModeRouter) && un.g >= p.E;
-        const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
-        const int KB = K / kTileK;
-        const int buf = static_cast<int>(ucount % static_cast<uint32_t>(p.nbuf));
-        const uint32_t bpar = (ucount / static_cast<uint32_t>(p.nbuf)) & 1u;
-        if (!mbar_wait(&tempty[buf], bpar ^ 1u, abort_flag, p.err, p.timeout_ns)) break;
-        tc_fence_after();
-        const uint32_t idesc = idesc_bf16_f32(kTileRows, un.n);
-        const uint32_t dcol = tmem_base + static_cast<uint32_t>(buf * NA * nmax);
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, p.timeout_ns)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // Token rows written by cp.async (generic proxy) are read by the
-          // tensor cores (async proxy).
-          if (MODE == kModeGateUp) fence_proxy_async_smem();
-          const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
-          const uint64_t bdesc = sw128_kmajor_desc(sbase + NA * kATileBytes);
-          uint64_t adesc[NA];
+      if constexpr (MODE == kModeRouter) {
+        // Router: the accumulator is drained every kRouterDrainKB k-blocks
+        // into fp32 registers by the epilogue, so no tensor-core accumulation
+        // chain is longer than 4 * kRouterDrainKB MMA steps.
+        uint32_t dc = 0;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+          const Unit un = get_unit<MODE>(p, u);
+          const int KB = p.d / kTileK;
+          const uint32_t idesc = idesc_bf16_f32(kTileRows, un.n);
+          uint32_t dcol = tmem_base;
+          for (int kb = 0; kb < KB; ++kb) {
+            const int sub = kb % kRouterDrainKB;
+            const int buf = static_cast<int>(dc % static_cast<uint32_t>(p.nbuf));
+            if (sub == 0) {
+              const uint32_t bpar = (dc / static_cast<uint32_t>(p.nbuf)) & 1u;
+              if (!mbar_wait(&tempty[buf], bpar ^ 1u, abort_flag, p.err, p.timeout_ns)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              dcol = tmem_base + static_cast<uint32_t>(buf * nmax);
+            }
+            if (!mbar_wait(&full[stage], phase, abort_flag, p.err, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+            const uint64_t adesc = sw128_kmajor_desc(sbase);
+            const uint64_t bdesc = sw128_kmajor_desc(sbase + kATileBytes);
 #pragma unroll
-          for (int a = 0; a < NA; ++a) adesc[a] = sw128_kmajor_desc(sbase + a * kATileBytes);
-#pragma unroll
-          for (int ks = 0; ks < kTileK / 16; ++ks) {
-#pragma unroll
-            for (int a = 0; a < NA; ++a)
-              tc_mma_bf16(dcol + static_cast<uint32_t>(a * nmax), adesc[a] + 2u * ks, bdesc + 2u * ks,
-                          idesc, (kb | ks) != 0 ? 1u : 0u);
-          }
-          any = true;
-          tc_commit(&empty[stage]);
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
+            for (int ks = 0; ks < kTileK / 16; ++ks)
+              tc_mma_bf16(dcol, adesc + 2u * ks, bdesc + 2u * ks, idesc, (sub | ks) != 0 ? 1u : 0u);
+            any = true;
+            tc_commit(&empty[stage]);
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            if (sub == kRouterDrainKB - 1 || kb == KB - 1) {
+              tc_commit(&tfull[buf]);
+              ++dc;
+            }
           }
         }
-        if (!ok) break;
-        tc_commit(&tfull[buf]);
-        ++ucount;
+      } else {
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+          const Unit un = get_unit<MODE>(p, u);
+          const bool sh = (MODE != kModeRouter) && un.g >= p.E;
+          const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
+          const int KB = K / kTileK;
+          const int buf = static_cast<int>(ucount % static_cast<uint32_t>(p.nbuf));
+          const uint32_t bpar = (ucount / static_cast<uint32_t>(p.nbuf)) & 1u;
+          if (!mbar_wait(&tempty[buf], bpar ^ 1u, abort_flag, p.err, p.timeout_ns)) break;
+          tc_fence_after();
+          const uint32_t idesc = idesc_bf16_f32(kTileRows, un.n);
+          const uint32_t dcol = tmem_base + static_cast<uint32_t>(buf * NA * nmax);
+          for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, p.err, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // Token rows written by cp.async (generic proxy) are read by the
+            // tensor cores (async proxy).
+            if (MODE == kModeGateUp) fence_proxy_async_smem();
+            const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+            const uint64_t bdesc = sw128_kmajor_desc(sbase + NA * kATileBytes);
+            uint64_t adesc[NA];
+#pragma unroll
+            for (int a = 0; a < NA; ++a) adesc[a] = sw128_kmajor_desc(sbase + a * kATileBytes);
+#pragma unroll
+            for (int ks = 0; ks < kTileK / 16; ++ks) {
+#pragma unroll
+              for (int a = 0; a < NA; ++a)
+                tc_mma_bf16(dcol + static_cast<uint32_t>(a * nmax), adesc[a] + 2u * ks, bdesc + 2u * ks,
+                            idesc, (kb | ks) != 0 ? 1u : 0u);
+            }
+            any = true;
+            tc_commit(&empty[stage]);
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          tc_commit(&tfull[buf]);
+          ++ucount;
+        }
       }
       // Leave no MMA in flight.
       if (any) {
@@ -296,94 +346,143 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                       // TMEM lane quarter this warp may read
     uint8_t* stg = epi + (warp - 2) * kEpiStageBytes;
-    uint32_t ucount = 0;
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
-      const Unit un = get_unit<MODE>(p, u);
-      const bool sh = (MODE != kModeRouter) && un.g >= p.E;
-      const int sidx = sh ? un.g - p.E : 0;
-      const int buf = static_cast<int>(ucount % static_cast<uint32_t>(p.nbuf));
-      const uint32_t bpar = (ucount / static_cast<uint32_t>(p.nbuf)) & 1u;
-      int got = 1;
-      if (lane == 0) got = mbar_wait(&tfull[buf], bpar, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
-      got = __shfl_sync(0xffffffffu, got, 0);
-      if (!got) break;
-      tc_fence_after();
-      const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * NA * nmax);
-      const int feat0 = un.wb * kTileRows + 32 * q;   // first weight row of this warp
-      const int wrows = (MODE == kModeRouter) ? p.E : (MODE == kModeGateUp ? (sh ? p.fs : p.f) : p.d);
-      if (feat0 < wrows) {
-        for (int c0 = 0; c0 < un.n; c0 += 16) {
-          uint32_t acc0[16], acc1[16];
-          tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c0), acc0);
-          if (NA == 2) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c0), acc1);
-          tmem_ld_wait();
-          if (MODE == kModeRouter) {
-            float* sf = reinterpret_cast<float*>(stg);
+    if constexpr (MODE == kModeRouter) {
+      // Router: sum the drained partial logits in fp32 registers, then write
+      // logits[t, e] (thread = expert row, column = token).
+      uint32_t dc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const Unit un = get_unit<MODE>(p, u);
+        const int KB = p.d / kTileK;
+        const int nd = (KB + kRouterDrainKB - 1) / kRouterDrainKB;
+        const int feat0 = un.wb * kTileRows + 32 * q;
+        const bool live = feat0 < p.E;
+        float acc[kRouterMaxN];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sf[i * 32 + lane] = __uint_as_float(acc0[i]);
+        for (int j = 0; j < kRouterMaxN; ++j) acc[j] = 0.0f;
+        for (int i = 0; i < nd; ++i) {
+          const int buf = static_cast<int>(dc % static_cast<uint32_t>(p.nbuf));
+          const uint32_t bpar = (dc / static_cast<uint32_t>(p.nbuf)) & 1u;
+          int got = 1;
+          if (lane == 0) got = mbar_wait(&tfull[buf], bpar, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (live) {
+            const uint32_t tb =
+                tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * nmax);
+            uint32_t v[4][16];
+#pragma unroll
+            for (int c = 0; c < kRouterMaxN / 16; ++c) tmem_ld_32x32b_x16(tb + 16u * c, v[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < kRouterMaxN / 16; ++c)
+#pragma unroll
+              for (int j = 0; j < 16; ++j) acc[16 * c + j] += __uint_as_float(v[c][j]);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+          ++dc;
+        }
+        if (!ok || !live) continue;
+        float* sf = reinterpret_cast<float*>(stg);
+#pragma unroll
+        for (int c = 0; c < kRouterMaxN / 16; ++c) {
+          if (16 * c < un.n) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sf[i * 32 + lane] = acc[16 * c + i];
             __syncwarp();
 #pragma unroll
             for (int rep = 0; rep < 4; ++rep) {
-              const int c = lane + 32 * rep;
-              const int tok = c >> 3, part = c & 7;
-              const int t = un.row0 + c0 + tok;
+              const int cc = lane + 32 * rep;
+              const int tok = cc >> 3, part = cc & 7;
+              const int t = un.row0 + 16 * c + tok;
               const int e = feat0 + part * 4;
               if (t < p.T) {
                 float* dst = reinterpret_cast<float*>(p.out_r) + static_cast<size_t>(t) * p.E + e;
-                const float4 v = *reinterpret_cast<const float4*>(sf + tok * 32 + part * 4);
+                const float4 vv = *reinterpret_cast<const float4*>(sf + tok * 32 + part * 4);
                 if ((p.E & 3) == 0 && e + 3 < p.E) {
-                  *reinterpret_cast<float4*>(dst) = v;
+                  *reinterpret_cast<float4*>(dst) = vv;
                 } else {
-                  if (e + 0 < p.E) dst[0] = v.x;
-                  if (e + 1 < p.E) dst[1] = v.y;
-                  if (e + 2 < p.E) dst[2] = v.z;
-                  if (e + 3 < p.E) dst[3] = v.w;
+                  if (e + 0 < p.E) dst[0] = vv.x;
+                  if (e + 1 < p.E) dst[1] = vv.y;
+                  if (e + 2 < p.E) dst[2] = vv.z;
+                  if (e + 3 < p.E) dst[3] = vv.w;
                 }
               }
-            }
-            __syncwarp();
-          } else {
-            __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
-            if (MODE == kModeGateUp) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float g = __uint_as_float(acc0[i]);
-                const float v = __uint_as_float(acc1[i]);
-                sb[i * 32 + lane] = __float2bfloat16_rn(silu_f(g) * v);
-              }
-            } else {
-              float wl = 1.0f;
-              if (!sh && lane < 16) wl = __ldg(p.roww + un.row0 + c0 + lane);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float w = __shfl_sync(0xffffffffu, wl, i);
-                sb[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(acc0[i]) * w);
-              }
-            }
-            __syncwarp();
-            const int ld = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
-            __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(sh ? p.out_s : p.out_r);
-            const size_t rbase = sh ? static_cast<size_t>(sidx) * p.Tp : 0;
-#pragma unroll
-            for (int rep = 0; rep < 2; ++rep) {
-              const int c = lane + 32 * rep;
-              const int tok = c >> 2, part = c & 3;
-              const uint4 v = *reinterpret_cast<const uint4*>(stg + tok * 64 + part * 16);
-              const size_t row = rbase + static_cast<size_t>(un.row0 + c0 + tok);
-              *reinterpret_cast<uint4*>(outp + row * ld + feat0 + part * 8) = v;
             }
             __syncwarp();
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
-      ++ucount;
+    } else {
+      uint32_t ucount = 0;
+      for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+        const Unit un = get_unit<MODE>(p, u);
+        const bool sh = (MODE != kModeRouter) && un.g >= p.E;
+        const int sidx = sh ? un.g - p.E : 0;
+        const int buf = static_cast<int>(ucount % static_cast<uint32_t>(p.nbuf));
+        const uint32_t bpar = (ucount / static_cast<uint32_t>(p.nbuf)) & 1u;
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&tfull[buf], bpar, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) break;
+        tc_fence_after();
+        const uint32_t tbase =
+            tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * NA * nmax);
+        const int feat0 = un.wb * kTileRows + 32 * q;   // first weight row of this warp
+        const int wrows = (MODE == kModeRouter) ? p.E : (MODE == kModeGateUp ? (sh ? p.fs : p.f) : p.d);
+        if (feat0 < wrows) {
+          for (int c0 = 0; c0 < un.n; c0 += 16) {
+            uint32_t acc0[16], acc1[16];
+            tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c0), acc0);
+            if (NA == 2) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c0), acc1);
+            tmem_ld_wait();
+            {
+              __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
+              if (MODE == kModeGateUp) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const float g = __uint_as_float(acc0[i]);
+                  const float v = __uint_as_float(acc1[i]);
+                  sb[i * 32 + lane] = __float2bfloat16_rn(silu_f(g) * v);
+                }
+              } else {
+                float wl = 1.0f;
+                if (!sh && lane < 16) wl = __ldg(p.roww + un.row0 + c0 + lane);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const float w = __shfl_sync(0xffffffffu, wl, i);
+                  sb[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(acc0[i]) * w);
+                }
+              }
+              __syncwarp();
+              const int ld = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
+              __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(sh ? p.out_s : p.out_r);
+              const size_t rbase = sh ? static_cast<size_t>(sidx) * p.Tp : 0;
+#pragma unroll
+              for (int rep = 0; rep < 2; ++rep) {
+                const int c = lane + 32 * rep;
+                const int tok = c >> 2, part = c & 3;
+                const uint4 v = *reinterpret_cast<const uint4*>(stg + tok * 64 + part * 16);
+                const size_t row = rbase + static_cast<size_t>(un.row0 + c0 + tok);
+                *reinterpret_cast<uint4*>(outp + row * ld + feat0 + part * 8) = v;
+              }
+              __syncwarp();
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+        ++ucount;
+      }
     }
-  }
-
+    }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
