@@ -169,7 +169,7 @@ int run_down(const Plan& p, const DeviceInfo& di, const void* Wd, const void* Ws
   int stages = 0;
   const size_t smem = gemm_smem_bytes(kModeDown, p.nmax2, &stages);
   g.stages = stages;
-  g.nbuf = (p.nmax2 <= 256) ? 2 : 1;
+  g.nbuf = (2 * p.nmax2 <= 256) ? 2 : 1;
   return launch_gemm(kModeDown, g, di.sms, smem, st);
 }
 
@@ -229,7 +229,7 @@ int make_plan(const moe_shape* s, Plan* p) {
   q.nwbE = ceil_div(E, kTileRows);
   q.nwb1 = ceil_div(f, kTileRows);
   q.nwb1s = S > 0 ? ceil_div(fs, kTileRows) : 0;
-  q.nwb2 = ceil_div(d, kTileRows);
+  q.nwb2 = ceil_div(d, 2 * kTileRows);      // down units cover 256 rows of W_down
   const double rows_per_expert = static_cast<double>(T) * k / E;
   q.nmax1 = pick_nmax(rows_per_expert);
   q.nmax2 = q.nmax1;

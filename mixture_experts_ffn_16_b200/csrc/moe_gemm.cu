@@ -35,12 +35,15 @@ namespace {
 
 constexpr int kGatherWarps = 4;                      // gate/up: warps that gather token rows
 constexpr int kGatherThreads = 32 * kGatherWarps;
+// Epilogue warps: 4 for the router (one per TMEM lane quarter), 8 for the
+// expert GEMMs (two per lane quarter, splitting the columns).
+__host__ __device__ constexpr int epi_warps_of(int mode) { return mode == kModeRouter ? 4 : 8; }
 __host__ __device__ constexpr int threads_of(int mode) {
-  return mode == kModeGateUp ? 192 + kGatherThreads : 192;
+  return 64 + 32 * epi_warps_of(mode) + (mode == kModeGateUp ? kGatherThreads : 0);
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kATileBytes = kTileRows * 128;   // 128 weight rows x 64 bf16
-constexpr int kEpiStageBytes = 2048;                 // per epilogue warp
+constexpr int kEpiBytes = 8192;                      // transpose staging, shared by the epilogue warps
 constexpr int kMaxStages = 8;
 constexpr int kSmemAlign = 1024;
 constexpr int kSmemTail = 512;                       // barriers, TMEM slot, abort flag
@@ -81,11 +84,17 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+// SiLU(z) = z * sigmoid(z) with the fast exponential and division; the
+// exponent is clamped so the denominator stays finite (|result| < 1e-32 there).
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(fminf(-z, 80.0f))); }
 
 template <int MODE>
 __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __grid_constant__ GemmParams p) {
-  constexpr int NA = (MODE == kModeGateUp) ? 2 : 1;   // A operands (accumulators) per unit
+  // A tiles (and accumulators) per unit: gate/up: the gate and the up tile of
+  // the same 128 rows; down: two consecutive 128-row blocks of W_down (a
+  // 256-row unit, so each token row loaded serves 256 outputs); router: one.
+  constexpr int NA = (MODE == kModeRouter) ? 1 : 2;
+  constexpr int kWbRows = (MODE == kModeDown) ? 2 * kTileRows : kTileRows;   // weight rows per unit
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + (kSmemAlign - 1)) & ~static_cast<uintptr_t>(kSmemAlign - 1));
@@ -93,7 +102,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
   const int S = p.stages;
   const uint32_t stage_bytes = NA * kATileBytes + static_cast<uint32_t>(nmax) * 128u;
   uint8_t* epi = smem + static_cast<size_t>(S) * stage_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(epi + 4 * kEpiStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi + kEpiBytes);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + kMaxTmemBufs;
@@ -112,7 +121,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
     }
     for (int b = 0; b < kMaxTmemBufs; ++b) {
       mbar_init(tfull + b, 1);
-      mbar_init(tempty + b, 4);
+      mbar_init(tempty + b, epi_warps_of(MODE));
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -165,7 +174,8 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
           mbar_arrive_expect_tx(&full[stage], tx_bytes);
 #pragma unroll
           for (int a = 0; a < NA; ++a)
-            tma_load_3d(sbase + a * kATileBytes, mA + a, fb, kb * kTileK, un.wb * kTileRows, a_c2);
+            tma_load_3d(sbase + a * kATileBytes, (MODE == kModeDown) ? mA : mA + a, fb, kb * kTileK,
+                        un.wb * kWbRows + ((MODE == kModeDown) ? a * kTileRows : 0), a_c2);
           if (MODE != kModeGateUp) {
             const uint32_t bbase = sbase + NA * kATileBytes;
             for (int i = 0; i < (un.n >> 4); ++i)
@@ -294,12 +304,12 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
       }
     }
     __syncwarp();
-  } else if (MODE == kModeGateUp && warp >= 6) {
+  } else if (MODE == kModeGateUp && warp >= 2 + epi_warps_of(MODE)) {
     // ------------------------------------------------------------ row gather
     // Thread g copies 16-byte chunk (g & 7) of rows (g >> 3) + 16 i of the
     // token tile, i < n / 16, into the 128-byte-swizzled slot: chunk c of row
     // r lands at r * 128 + ((c ^ (r & 7)) * 16).
-    const int g = threadIdx.x - 192;
+    const int g = threadIdx.x - 32 * (2 + epi_warps_of(MODE));
     const int part = g & 7;
     const int r0 = g >> 3;
     int stage = 0;
@@ -342,10 +352,10 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
       }
     }
     cp_async_wait_all();
-  } else if (warp >= 2 && warp < 6) {
+  } else if (warp >= 2 && warp < 2 + epi_warps_of(MODE)) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                       // TMEM lane quarter this warp may read
-    uint8_t* stg = epi + (warp - 2) * kEpiStageBytes;
+    uint8_t* stg = epi + (warp - 2) * (kEpiBytes / epi_warps_of(MODE));
     if constexpr (MODE == kModeRouter) {
       // Router: sum the drained partial logits in fp32 registers, then write
       // logits[t, e] (thread = expert row, column = token).
@@ -432,48 +442,76 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) break;
         tc_fence_after();
-        const uint32_t tbase =
-            tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * NA * nmax);
-        const int feat0 = un.wb * kTileRows + 32 * q;   // first weight row of this warp
-        const int wrows = (MODE == kModeRouter) ? p.E : (MODE == kModeGateUp ? (sh ? p.fs : p.f) : p.d);
+        // gate/up: warps (q, half) take column blocks half*16, half*16 + 32, ...
+        // of both accumulators; down: warps (q, h) take every column of
+        // accumulator h (weight rows wb*256 + h*128 ...).
+        const int half = (MODE == kModeGateUp) ? ((warp - 2) >> 2) : 0;
+        const int h = (MODE == kModeDown) ? ((warp - 2) >> 2) : 0;
+        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                               static_cast<uint32_t>(buf * NA * nmax + h * nmax);
+        const int feat0 = un.wb * kWbRows + h * kTileRows + 32 * q;   // first weight row of this warp
+        const int wrows = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
         if (feat0 < wrows) {
-          for (int c0 = 0; c0 < un.n; c0 += 16) {
-            uint32_t acc0[16], acc1[16];
-            tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c0), acc0);
-            if (NA == 2) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c0), acc1);
-            tmem_ld_wait();
-            {
-              __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
-              if (MODE == kModeGateUp) {
+          const int ld = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
+          __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(sh ? p.out_s : p.out_r);
+          const size_t rbase = (sh ? static_cast<size_t>(sidx) * p.Tp : 0) + static_cast<size_t>(un.row0);
+          // 16 columns: fp32 math, bf16, transpose through shared memory,
+          // 16-byte stores of 64-byte row segments.
+          auto emit = [&](const uint32_t (&A)[16], const uint32_t (&B)[16], int c) {
+            __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
+            if (MODE == kModeGateUp) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                  const float g = __uint_as_float(acc0[i]);
-                  const float v = __uint_as_float(acc1[i]);
-                  sb[i * 32 + lane] = __float2bfloat16_rn(silu_f(g) * v);
-                }
-              } else {
-                float wl = 1.0f;
-                if (!sh && lane < 16) wl = __ldg(p.roww + un.row0 + c0 + lane);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                  const float w = __shfl_sync(0xffffffffu, wl, i);
-                  sb[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(acc0[i]) * w);
-                }
+              for (int i = 0; i < 16; ++i) {
+                const float g = __uint_as_float(A[i]);
+                const float v = __uint_as_float(B[i]);
+                sb[i * 32 + lane] = __float2bfloat16_rn(silu_f(g) * v);
               }
-              __syncwarp();
-              const int ld = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
-              __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(sh ? p.out_s : p.out_r);
-              const size_t rbase = sh ? static_cast<size_t>(sidx) * p.Tp : 0;
+            } else {
+              float wl = 1.0f;
+              if (!sh && lane < 16) wl = __ldg(p.roww + un.row0 + c + lane);
 #pragma unroll
-              for (int rep = 0; rep < 2; ++rep) {
-                const int c = lane + 32 * rep;
-                const int tok = c >> 2, part = c & 3;
-                const uint4 v = *reinterpret_cast<const uint4*>(stg + tok * 64 + part * 16);
-                const size_t row = rbase + static_cast<size_t>(un.row0 + c0 + tok);
-                *reinterpret_cast<uint4*>(outp + row * ld + feat0 + part * 8) = v;
+              for (int i = 0; i < 16; ++i) {
+                const float w = __shfl_sync(0xffffffffu, wl, i);
+                sb[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(A[i]) * w);
               }
-              __syncwarp();
             }
+            __syncwarp();
+#pragma unroll
+            for (int rep = 0; rep < 2; ++rep) {
+              const int cc = lane + 32 * rep;
+              const int tok = cc >> 2, part = cc & 3;
+              const uint4 v = *reinterpret_cast<const uint4*>(stg + tok * 64 + part * 16);
+              *reinterpret_cast<uint4*>(outp + (rbase + c + tok) * ld + feat0 + part * 8) = v;
+            }
+            __syncwarp();
+          };
+          // Two register sets: the TMEM load of the next 16 columns is in
+          // flight while the current ones are converted and stored.  This
+          // warp takes column blocks half*16, half*16 + 32, ...
+          constexpr int kStep = (MODE == kModeGateUp) ? 32 : 16;
+          uint32_t a0[16], b0[16], a1[16], b1[16];
+          int c0 = 16 * half;
+          if (c0 < un.n) {
+            tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c0), a0);
+            if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c0), b0);
+          }
+          while (c0 < un.n) {
+            tmem_ld_wait();
+            const int c1 = c0 + kStep;
+            if (c1 < un.n) {
+              tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c1), a1);
+              if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c1), b1);
+            }
+            emit(a0, b0, c0);
+            if (c1 >= un.n) break;
+            tmem_ld_wait();
+            const int c2 = c1 + kStep;
+            if (c2 < un.n) {
+              tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c2), a0);
+              if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c2), b0);
+            }
+            emit(a1, b1, c1);
+            c0 = c2;
           }
         }
         tc_fence_before();
@@ -494,9 +532,9 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
 }  // namespace
 
 size_t gemm_smem_bytes(int mode, int nmax, int* stages) {
-  const int NA = (mode == kModeGateUp) ? 2 : 1;
+  const int NA = (mode == kModeRouter) ? 1 : 2;
   const size_t stage_bytes = NA * static_cast<size_t>(kATileBytes) + static_cast<size_t>(nmax) * 128;
-  const size_t fixed = kSmemAlign + 4 * kEpiStageBytes + kSmemTail;
+  const size_t fixed = kSmemAlign + kEpiBytes + kSmemTail;
   const size_t budget = 232448;   // sm_100 opt-in maximum per block
   int s = static_cast<int>((budget - fixed) / stage_bytes);
   if (s > kMaxStages) s = kMaxStages;

@@ -8,7 +8,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/moe.h"
+#include "moe.h"
 
 namespace moe {
 
@@ -35,7 +35,7 @@ struct Plan {
   int nwbE;        // 128-row blocks of E
   int nwb1;        // 128-row blocks of f
   int nwb1s;       // 128-row blocks of fs
-  int nwb2;        // 128-row blocks of d
+  int nwb2;        // 256-row blocks of d (down-projection units)
   int router_units;
   int U1cap, U2cap;
   int shared_units1, shared_units2;

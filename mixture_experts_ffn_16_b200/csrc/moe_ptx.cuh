@@ -65,6 +65,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended (not spinning) for up to
+// `hint_ns` nanoseconds while the phase is still pending.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of parity `parity` to complete.  Gives up when
 // another role of the block has already given up (*abort != 0) or when
 // `timeout_ns` has passed; then sets *abort, records kDevErrTimeout in *err
@@ -75,8 +89,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(a, parity)) return true;
-    if ((it & 31u) == 0) {
+    if (mbar_try_wait_sleep(a, parity, 20000u)) return true;
+    if ((it & 7u) == 0) {
       if (*abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
         *abort = 1;
