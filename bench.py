@@ -127,12 +127,19 @@ def dist_setup(n_gpus):
 
 
 def max_over_ranks(v, world):
+    """Max of a per-rank time over all ranks (NCCL on GPUs, gloo on CPU)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(cfg, rank):
+    """Each replica draws its own token batch and weights (weak scaling)."""
+    return cfg.seed + 1000 * rank
 
 
 def barrier(world):
@@ -213,7 +220,7 @@ def run_ours(args, cfg):
     world, rank, local = dist_setup(args.gpus)
     api.load()
     dev = torch.device("cuda", local if world > 1 else 0)
-    inp = make_inputs(cfg, device=dev, seed=cfg.seed + 1000 * rank)
+    inp = make_inputs(cfg, device=dev, seed=replica_seed(cfg, rank))
     layer = api.MoELayer(cfg, inp, device=dev)
     stream = torch.cuda.current_stream(dev)
     s = layer.shape
