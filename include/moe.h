@@ -67,6 +67,7 @@ extern "C" {
 #define MOE_ERR_WORKSPACE      -3   /* workspace missing, misaligned or smaller than moe_workspace_bytes */
 #define MOE_ERR_CUDA           -4   /* a CUDA runtime / driver call or a launch failed */
 #define MOE_ERR_DEVICE_TIMEOUT -5   /* a bounded device-side wait ran out (reported by moe_device_status) */
+#define MOE_ERR_SCRATCH_LIMIT  -6   /* moe_route_noalloc: T * E fp32 logits exceed its built-in 16 MiB scratch */
 
 #define MOE_SCORE_SOFTMAX       0   /* s = softmax(l) over all E experts; expert_bias ignored */
 #define MOE_SCORE_SIGMOID       1   /* s = 1/(1+exp(-l)) */
@@ -197,6 +198,31 @@ MOE_API int moe_workspace_region(const moe_shape *shape, int region, size_t *off
  * call on this workspace (since the last moe_route) gave up a bounded wait,
  * MOE_ERR_CUDA if the stream reports an error, else MOE_OK. */
 MOE_API int moe_device_status(const void *workspace, moe_stream_t stream);
+
+/* Routing (the moe_route step) for callers that cannot allocate device
+ * memory, such as an inference-engine plugin whose per-call hook may not
+ * allocate, or a process whose device memory is reserved up front by another
+ * allocator.  The pages have no counterpart: this is an integration variant,
+ * not part of the method.
+ *   Same arguments and results as moe_route, without the workspace: the fp32
+ *   logits live in a 16 MiB array compiled into this library, which every GPU
+ *   that loads the library holds until the process exits.  Shapes with
+ *   T * E * 4 bytes > 16 MiB (T * E > 4,194,304) return MOE_ERR_SCRATCH_LIMIT
+ *   and enqueue nothing.  x, W_router, expert_bias, topk_idx and topk_w are
+ *   the caller's, as for moe_route.  Allocates nothing (no cudaMalloc /
+ *   cudaFree) on any call.
+ *   The first call on a device looks up the array's device address (a CUDA
+ *   runtime query, once per device, with that device current); make that
+ *   first call before any stream capture.
+ *   Every call uses the same array: two calls that overlap on the GPU (on
+ *   different streams, or from different threads without ordering) race and
+ *   give undefined results.  The array keeps the last call's contents; the
+ *   call clears what must start at zero itself.
+ *   A bounded device wait that runs out is recorded only inside that array:
+ *   moe_device_status cannot report it for this entry point. */
+MOE_API int moe_route_noalloc(const moe_shape *shape, const void *x, const void *W_router,
+                              const float *expert_bias, int score_fn, int norm_topk, float route_scale,
+                              int32_t *topk_idx, float *topk_w, moe_stream_t stream);
 
 /* Self-test of the bounded-wait machinery: launches one block that waits on a
  * shared-memory barrier which nothing ever completes, for at most timeout_ns

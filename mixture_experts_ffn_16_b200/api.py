@@ -22,6 +22,7 @@ MOE_ERR_UNSUPPORTED = -2
 MOE_ERR_WORKSPACE = -3
 MOE_ERR_CUDA = -4
 MOE_ERR_DEVICE_TIMEOUT = -5
+MOE_ERR_SCRATCH_LIMIT = -6
 
 SCORE_FNS = {"softmax": 0, "sigmoid": 1, "sqrt_softplus": 2}
 
@@ -30,7 +31,8 @@ WS_REGIONS = {"logits": 0, "counts": 1, "offsets": 2, "perm": 3, "row_w": 4, "in
 
 EXPORTED = ["moe_version", "moe_status_string", "moe_workspace_bytes", "moe_forward",
             "moe_forward_host", "moe_route", "moe_permute", "moe_expert_gate_up", "moe_expert_down",
-            "moe_combine", "moe_workspace_region", "moe_device_status", "moe_debug_wait_timeout"]
+            "moe_combine", "moe_workspace_region", "moe_device_status", "moe_debug_wait_timeout",
+            "moe_route_noalloc"]
 
 
 class MoEError(RuntimeError):
@@ -86,6 +88,8 @@ def load():
     lib.moe_device_status.argtypes = [P, P]
     lib.moe_debug_wait_timeout.restype = I
     lib.moe_debug_wait_timeout.argtypes = [P, SZ, ctypes.c_uint64, P]
+    lib.moe_route_noalloc.restype = I
+    lib.moe_route_noalloc.argtypes = [SH, P, P, P, I, I, ctypes.c_float, P, P, P]
     _lib = lib
     return lib
 
@@ -219,6 +223,21 @@ def moe_route(shape, x, W_router, expert_bias, score_fn, norm_topk, route_scale,
         _p(topk_w, torch.float32, (T, k), "topk_w"), _p(workspace, torch.uint8, None, "workspace"),
         workspace.numel(), _stream(stream))
     _check(st, "moe_route")
+
+
+def moe_route_noalloc(shape, x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w,
+                      stream=None):
+    """moe_route without a workspace, for callers that cannot allocate device
+    memory (the library's built-in 16 MiB scratch holds the logits; T * E must
+    not exceed 4,194,304).  Calls that overlap on the GPU race."""
+    T, d, E, k = shape.T, shape.d_model, shape.E, shape.k
+    bf = torch.bfloat16
+    st = load().moe_route_noalloc(
+        ctypes.byref(shape), _p(x, bf, (T, d), "x"), _p(W_router, bf, (E, d), "W_router"),
+        _p(expert_bias, torch.float32, (E,), "expert_bias"), _score(score_fn), int(bool(norm_topk)),
+        float(route_scale), _p(topk_idx, torch.int32, (T, k), "topk_idx"),
+        _p(topk_w, torch.float32, (T, k), "topk_w"), _stream(stream))
+    _check(st, "moe_route_noalloc")
 
 
 def moe_permute(shape, topk_idx, topk_w, workspace, stream=None):

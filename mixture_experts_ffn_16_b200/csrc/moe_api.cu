@@ -315,6 +315,8 @@ const char* moe_status_string(int status) {
     case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA call or kernel launch failed";
     case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a bounded device-side wait ran out";
+    case MOE_ERR_SCRATCH_LIMIT:
+      return "MOE_ERR_SCRATCH_LIMIT: T * E fp32 logits exceed the 16 MiB built-in scratch of moe_route_noalloc";
     default: return "unknown status";
   }
 }
@@ -498,3 +500,81 @@ int moe_debug_wait_timeout(void* workspace, size_t workspace_bytes, uint64_t tim
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Routing for callers that cannot allocate device memory.
+//
+// moe_route needs a caller-provided workspace for the fp32 logits between the
+// router GEMM and the top-k kernel.  Some callers cannot hand one over: an
+// inference-engine plugin whose per-call hook may not allocate, or a service
+// whose device memory is entirely reserved up front by another allocator.
+// moe_route_noalloc runs the same two kernels with that scratch in a
+// fixed-size array compiled into this library instead.
+namespace moe {
+namespace {
+
+constexpr size_t kNoAllocHeaderBytes = 256;                 // device error word, padded
+constexpr size_t kNoAllocLogitBytes = size_t(16) << 20;     // fp32 logits: T * E <= 4,194,304
+static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocHeaderBytes + kNoAllocLogitBytes];
+
+char* g_route_scratch_dev[64];    // device address of g_route_scratch, per device
+int g_route_scratch_ready[64];
+
+// The host-side name g_route_scratch is not a device address: look up the
+// device address once per device (with that device current) and reuse it.
+int route_scratch_address(char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  if (!g_route_scratch_ready[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_route_scratch) != cudaSuccess || ptr == nullptr) return MOE_ERR_CUDA;
+    g_route_scratch_dev[dev] = static_cast<char*>(ptr);
+    g_route_scratch_ready[dev] = 1;
+  }
+  *out = g_route_scratch_dev[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_route_noalloc(const moe_shape* shape, const void* x, const void* W_router,
+                                 const float* expert_bias, int score_fn, int norm_topk, float route_scale,
+                                 int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_route_args(x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w)) != MOE_OK)
+    return rc;
+  if (static_cast<size_t>(p.T) * static_cast<size_t>(p.E) * sizeof(float) > kNoAllocLogitBytes)
+    return MOE_ERR_SCRATCH_LIMIT;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  char* scratch = nullptr;
+  if ((rc = route_scratch_address(&scratch)) != MOE_OK) return rc;
+  cudaStream_t st = as_stream(stream);
+  uint32_t* err = reinterpret_cast<uint32_t*>(scratch);
+  float* logits = reinterpret_cast<float*>(scratch + kNoAllocHeaderBytes);
+  // The array keeps the previous call's contents: the error word must start at zero.
+  if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+  GemmParams g;
+  std::memset(&g, 0, sizeof g);
+  if (!map_weights(&g.mapA[0], W_router, p.d, p.E, 1) || !map_rows(&g.mapB[0], x, p.d, p.T, kRowPad))
+    return MOE_ERR_CUDA;
+  g.mapA[1] = g.mapA[2] = g.mapA[3] = g.mapA[0];
+  g.mapB[1] = g.mapB[0];
+  g.num_units_host = p.router_units;
+  g.out_r = logits;
+  g.err = err;
+  g.T = p.T; g.Tp = p.Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
+  g.nmax = p.nmax_r;
+  g.router_nwb = p.nwbE;
+  g.timeout_ns = kWaitTimeoutNs;
+  int stages = 0;
+  const size_t smem = gemm_smem_bytes(kModeRouter, p.nmax_r, &stages);
+  g.stages = stages;
+  g.nbuf = 512 / p.nmax_r < 8 ? 512 / p.nmax_r : 8;
+  const int grid = p.router_units < di.sms ? p.router_units : di.sms;
+  if ((rc = launch_gemm(kModeRouter, g, grid, smem, st)) != MOE_OK) return rc;
+  return launch_topk(logits, expert_bias, p.T, p.E, p.k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
+}
