@@ -33,7 +33,8 @@ if ROOT not in sys.path:
 
 from mixture_experts_ffn_16_b200 import api  # noqa: E402
 from mixture_experts_ffn_16_b200.inputs import CONFIGS, make_inputs, oracle_args  # noqa: E402
-from mixture_experts_ffn_16_b200.roofline import block_cost, kernel_costs, measured_peaks  # noqa: E402
+from mixture_experts_ffn_16_b200.roofline import (block_cost, kernel_costs, measured_peaks,  # noqa: E402
+                                                  measured_traffic)
 
 METRIC = "MoE-layer tokens/sec at 1 B200; % bf16 tensor peak (prefill) / % HBM BW (decode)"
 STAGES = ["route", "permute", "gate_up", "down", "combine"]
@@ -318,7 +319,7 @@ def run_ours(args, cfg):
     else:
         roof = {"bound": "hbm", "achieved": by / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(cfg.name, dom)
     roof["kernel"] = dom
     roof["algorithmic_bytes"] = by
     roof["algorithmic_flops"] = fl

@@ -48,8 +48,7 @@ bool map_weights(CUtensorMap* m, const void* ptr, int K, int rows, int G) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Token-row source [rows, K] bf16, 128-byte swizzle.  box_rows = 1 for the
-// gather4 loads (one row high box), kRowPad for tiled loads of 16 rows.
+// Token-row source [rows, K] bf16, 128-byte swizzle, box of box_rows rows.
 bool map_rows(CUtensorMap* m, const void* ptr, int K, int rows, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -61,6 +60,17 @@ bool map_rows(CUtensorMap* m, const void* ptr, int K, int rows, int box_rows) {
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             box_rows == 1 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The four token-row maps of one source: boxes of 16, 32, 64 and 128 rows.
+bool map_rows_set(CUtensorMap (&m)[4], const void* ptr, int K, int rows) {
+  for (int b = 0; b < 4; ++b)
+    if (!map_rows(&m[b], ptr, K, rows, kRowPad << b)) return false;
+  return true;
+}
+
+void copy_set(CUtensorMap (&dst)[4], const CUtensorMap (&src)[4]) {
+  for (int b = 0; b < 4; ++b) dst[b] = src[b];
 }
 
 int pick_nmax(double rows_per_expert) {
@@ -89,10 +99,10 @@ int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_
   if (cudaMemsetAsync(ws + p.err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
   GemmParams g;
   std::memset(&g, 0, sizeof g);
-  if (!map_weights(&g.mapA[0], W_router, p.d, p.E, 1) || !map_rows(&g.mapB[0], x, p.d, p.T, kRowPad))
+  if (!map_weights(&g.mapA[0], W_router, p.d, p.E, 1) || !map_rows_set(g.mapB[0], x, p.d, p.T))
     return MOE_ERR_CUDA;
   g.mapA[1] = g.mapA[2] = g.mapA[3] = g.mapA[0];
-  g.mapB[1] = g.mapB[0];
+  copy_set(g.mapB[1], g.mapB[0]);
   g.num_units_host = p.router_units;
   g.out_r = ws + p.logits;
   g.err = reinterpret_cast<uint32_t*>(ws + p.err);
@@ -116,7 +126,7 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* 
   GemmParams g;
   std::memset(&g, 0, sizeof g);
   if (!map_weights(&g.mapA[0], Wg, p.d, p.f, p.E) || !map_weights(&g.mapA[1], Wu, p.d, p.f, p.E) ||
-      !map_rows(&g.mapB[0], x, p.d, p.T, 1))
+      !map_rows_set(g.mapB[0], x, p.d, p.T))
     return MOE_ERR_CUDA;
   if (p.S > 0) {
     if (!map_weights(&g.mapA[2], Wsg, p.d, p.fs, p.S) || !map_weights(&g.mapA[3], Wsu, p.d, p.fs, p.S))
@@ -125,7 +135,7 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* 
     g.mapA[2] = g.mapA[0];
     g.mapA[3] = g.mapA[1];
   }
-  g.mapB[1] = g.mapB[0];
+  copy_set(g.mapB[1], g.mapB[0]);
   g.units = reinterpret_cast<const int4*>(ws + p.units1);
   g.num_units_dev = reinterpret_cast<const int*>(ws + p.nunits);
   g.perm = reinterpret_cast<const int*>(ws + p.perm);
@@ -137,23 +147,28 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* 
   g.nmax = p.nmax1;
   g.timeout_ns = kWaitTimeoutNs;
   int stages = 0;
+  g.nbuf = (2 * p.nmax1 <= 256) ? 2 : 1;
+  if (p.pair1) {
+    const size_t smem = gemm_pair_smem_bytes(kModeGateUp, p.nmax1, &stages);
+    g.stages = stages;
+    return launch_gemm_pair(kModeGateUp, g, di.sms, smem, st);
+  }
   const size_t smem = gemm_smem_bytes(kModeGateUp, p.nmax1, &stages);
   g.stages = stages;
-  g.nbuf = (2 * p.nmax1 <= 256) ? 2 : 1;
   return launch_gemm(kModeGateUp, g, di.sms, smem, st);
 }
 
 int run_down(const Plan& p, const DeviceInfo& di, const void* Wd, const void* Wsd, char* ws, cudaStream_t st) {
   GemmParams g;
   std::memset(&g, 0, sizeof g);
-  if (!map_weights(&g.mapA[0], Wd, p.f, p.d, p.E) || !map_rows(&g.mapB[0], ws + p.Hr, p.f, p.Rcap, kRowPad))
+  if (!map_weights(&g.mapA[0], Wd, p.f, p.d, p.E) || !map_rows_set(g.mapB[0], ws + p.Hr, p.f, p.Rcap))
     return MOE_ERR_CUDA;
   if (p.S > 0) {
-    if (!map_weights(&g.mapA[2], Wsd, p.fs, p.d, p.S) || !map_rows(&g.mapB[1], ws + p.Hs, p.fs, p.S * p.Tp, kRowPad))
+    if (!map_weights(&g.mapA[2], Wsd, p.fs, p.d, p.S) || !map_rows_set(g.mapB[1], ws + p.Hs, p.fs, p.S * p.Tp))
       return MOE_ERR_CUDA;
   } else {
     g.mapA[2] = g.mapA[0];
-    g.mapB[1] = g.mapB[0];
+    copy_set(g.mapB[1], g.mapB[0]);
   }
   g.mapA[1] = g.mapA[0];
   g.mapA[3] = g.mapA[2];
@@ -167,9 +182,15 @@ int run_down(const Plan& p, const DeviceInfo& di, const void* Wd, const void* Ws
   g.nmax = p.nmax2;
   g.timeout_ns = kWaitTimeoutNs;
   int stages = 0;
+  if (p.pair2) {
+    g.nbuf = (p.nmax2 <= 256) ? 2 : 1;          // one accumulator per CTA
+    const size_t smem = gemm_pair_smem_bytes(kModeDown, p.nmax2, &stages);
+    g.stages = stages;
+    return launch_gemm_pair(kModeDown, g, di.sms, smem, st);
+  }
+  g.nbuf = (2 * p.nmax2 <= 256) ? 2 : 1;
   const size_t smem = gemm_smem_bytes(kModeDown, p.nmax2, &stages);
   g.stages = stages;
-  g.nbuf = (2 * p.nmax2 <= 256) ? 2 : 1;
   return launch_gemm(kModeDown, g, di.sms, smem, st);
 }
 
@@ -219,20 +240,29 @@ int make_plan(const moe_shape* s, Plan* p) {
   if (E > kMaxE || k > kMaxK || S > kMaxShared) return MOE_ERR_UNSUPPORTED;
   if (d % 64 || f % 64 || (S > 0 && fs % 64)) return MOE_ERR_UNSUPPORTED;
   if (T > (1 << 22) || d > (1 << 16) || f > (1 << 16) || fs > (1 << 16)) return MOE_ERR_UNSUPPORTED;
-  if (static_cast<long long>(T) * k + static_cast<long long>(E) * kRowPad > (1ll << 30)) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * k + static_cast<long long>(E) * 2 * kRowPad > (1ll << 30)) return MOE_ERR_UNSUPPORTED;
   Plan q;
   std::memset(&q, 0, sizeof q);
   q.T = T; q.d = d; q.E = E; q.k = k; q.f = f; q.S = S; q.fs = fs;
-  q.Tp = ceil_div(T, kRowPad) * kRowPad;
-  q.Rcap = ceil_div(T * k + E * (kRowPad - 1), kRowPad) * kRowPad;
-  q.nb = ceil_div(T, kPermBlock);
-  q.nwbE = ceil_div(E, kTileRows);
-  q.nwb1 = ceil_div(f, kTileRows);
-  q.nwb1s = S > 0 ? ceil_div(fs, kTileRows) : 0;
-  q.nwb2 = ceil_div(d, 2 * kTileRows);      // down units cover 256 rows of W_down
   const double rows_per_expert = static_cast<double>(T) * k / E;
   q.nmax1 = pick_nmax(rows_per_expert);
   q.nmax2 = q.nmax1;
+  // Experts of 256+ rows on average: the gate/up GEMM runs on CTA pairs,
+  // each CTA loading half of every token tile (runs then come in multiples of
+  // 32).  Below that, and for the down GEMM (measured), the pair's cross-CTA
+  // handshakes cost more than the halved token loads save.
+  q.pair1 = (q.nmax1 >= 64 && rows_per_expert >= 256.0) ? 1 : 0;
+  q.pair2 = 0;
+  q.rowpad = (q.pair1 || q.pair2) ? 2 * kRowPad : kRowPad;
+  q.Tp = ceil_div(T, q.rowpad) * q.rowpad;
+  q.Rcap = ceil_div(T * k + E * (q.rowpad - 1), q.rowpad) * q.rowpad;
+  q.nb = ceil_div(T, kPermBlock);
+  q.nwbE = ceil_div(E, kTileRows);
+  const int rows1 = q.pair1 ? 2 * kTileRows : kTileRows;   // weight rows per gate/up unit
+  const int rows2 = 2 * kTileRows;                          // weight rows per down unit
+  q.nwb1 = ceil_div(f, rows1);
+  q.nwb1s = S > 0 ? ceil_div(fs, rows1) : 0;
+  q.nwb2 = ceil_div(d, rows2);
   // Router: runs of up to 64 tokens (their fp32 logit sums live in registers);
   // narrower runs only when that leaves most SMs of a B200 idle.
   q.nmax_r = 16;
@@ -559,10 +589,10 @@ extern "C" int moe_route_noalloc(const moe_shape* shape, const void* x, const vo
   if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
   GemmParams g;
   std::memset(&g, 0, sizeof g);
-  if (!map_weights(&g.mapA[0], W_router, p.d, p.E, 1) || !map_rows(&g.mapB[0], x, p.d, p.T, kRowPad))
+  if (!map_weights(&g.mapA[0], W_router, p.d, p.E, 1) || !map_rows_set(g.mapB[0], x, p.d, p.T))
     return MOE_ERR_CUDA;
   g.mapA[1] = g.mapA[2] = g.mapA[3] = g.mapA[0];
-  g.mapB[1] = g.mapB[0];
+  copy_set(g.mapB[1], g.mapB[0]);
   g.num_units_host = p.router_units;
   g.out_r = logits;
   g.err = err;

@@ -84,6 +84,14 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
+// v[j] for a run-time j in [0, 8), without indexing the array dynamically.
+__device__ __forceinline__ float pick8(const float (&v)[8], int j) {
+  float r = v[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) r = (i == j) ? v[i] : r;
+  return r;
+}
+
 // SiLU(z) = z * sigmoid(z) with the fast exponential and division; the
 // exponent is clamped so the denominator stays finite (|result| < 1e-32 there).
 __device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(fminf(-z, 80.0f))); }
@@ -129,8 +137,8 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
   }
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < 2 * NA; ++i) prefetch_tensormap(&p.mapA[i]);
-    prefetch_tensormap(&p.mapB[0]);
-    if (MODE == kModeDown) prefetch_tensormap(&p.mapB[1]);
+    if (MODE != kModeGateUp)
+      for (int i = 0; i < 4; ++i) prefetch_tensormap(&p.mapB[0][i]);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -155,7 +163,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
       const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
       const int KB = K / kTileK;
       const CUtensorMap* mA = &p.mapA[sh ? 2 : 0];
-      const CUtensorMap* mB = &p.mapB[(MODE == kModeDown && sh) ? 1 : 0];
+      const CUtensorMap* mB = p.mapB[(MODE == kModeDown && sh) ? 1 : 0];
       const int a_c2 = (MODE == kModeRouter) ? 0 : (sh ? sidx : un.g);
       // Router / down: the unit's rows are contiguous in the source; first row:
       const int brow0 = (MODE == kModeDown && sh) ? sidx * p.Tp + un.row0 : un.row0;
@@ -176,11 +184,8 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
           for (int a = 0; a < NA; ++a)
             tma_load_3d(sbase + a * kATileBytes, (MODE == kModeDown) ? mA : mA + a, fb, kb * kTileK,
                         un.wb * kWbRows + ((MODE == kModeDown) ? a * kTileRows : 0), a_c2);
-          if (MODE != kModeGateUp) {
-            const uint32_t bbase = sbase + NA * kATileBytes;
-            for (int i = 0; i < (un.n >> 4); ++i)
-              tma_load_2d(bbase + i * 2048u, mB, fb, kb * kTileK, brow0 + 16 * i);
-          }
+          if (MODE != kModeGateUp)
+            tma_load_rows<false>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, un.n);
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -437,6 +442,14 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
         const int sidx = sh ? un.g - p.E : 0;
         const int buf = static_cast<int>(ucount % static_cast<uint32_t>(p.nbuf));
         const uint32_t bpar = (ucount / static_cast<uint32_t>(p.nbuf)) & 1u;
+        // down: combine weights of the unit's rows, fetched before the wait
+        // (lane l of register j holds the weight of column 32 j + l)
+        float wreg[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = 32 * j + lane;
+          wreg[j] = (MODE == kModeDown && !sh && c < un.n) ? __ldg(p.roww + un.row0 + c) : 1.0f;
+        }
         int got = 1;
         if (lane == 0) got = mbar_wait(&tfull[buf], bpar, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
         got = __shfl_sync(0xffffffffu, got, 0);
@@ -457,7 +470,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
           const size_t rbase = (sh ? static_cast<size_t>(sidx) * p.Tp : 0) + static_cast<size_t>(un.row0);
           // 16 columns: fp32 math, bf16, transpose through shared memory,
           // 16-byte stores of 64-byte row segments.
-          auto emit = [&](const uint32_t (&A)[16], const uint32_t (&B)[16], int c) {
+          auto emit = [&](const uint32_t (&A)[16], const uint32_t (&B)[16], int c, float wsel) {
             __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
             if (MODE == kModeGateUp) {
 #pragma unroll
@@ -467,11 +480,9 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
                 sb[i * 32 + lane] = __float2bfloat16_rn(silu_f(g) * v);
               }
             } else {
-              float wl = 1.0f;
-              if (!sh && lane < 16) wl = __ldg(p.roww + un.row0 + c + lane);
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const float w = __shfl_sync(0xffffffffu, wl, i);
+                const float w = __shfl_sync(0xffffffffu, wsel, (c + i) & 31);
                 sb[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(A[i]) * w);
               }
             }
@@ -502,7 +513,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
               tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c1), a1);
               if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c1), b1);
             }
-            emit(a0, b0, c0);
+            emit(a0, b0, c0, MODE == kModeDown ? pick8(wreg, c0 >> 5) : 1.0f);
             if (c1 >= un.n) break;
             tmem_ld_wait();
             const int c2 = c1 + kStep;
@@ -510,7 +521,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
               tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c2), a0);
               if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c2), b0);
             }
-            emit(a1, b1, c1);
+            emit(a1, b1, c1, MODE == kModeDown ? pick8(wreg, c1 >> 5) : 1.0f);
             c0 = c2;
           }
         }
@@ -529,6 +540,364 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
   }
 }
 
+
+// ===========================================================================
+// CTA-pair version of the expert GEMMs (tcgen05 cta_group::2).
+//
+// A cluster of two CTAs (on the two SMs of a TPC) works on one pair-unit
+// {group g, weight block wb, first row row0, n tokens}.  Every MMA has M = 256:
+// CTA r supplies weight rows [.. + r*128, +128) and token rows
+// [r*n/2, (r+1)*n/2) of the tile, and receives its 128 rows of every output
+// column in its own tensor memory.  Each CTA therefore loads half of the token
+// tile that a single CTA would: the token bytes that stream into the SMs are
+// halved for the same weight bytes.
+//   gate/up : wb = 256-row block of f; A tiles per CTA: gate rows, up rows.
+//   down    : wb = 512-row block of d; A tiles per CTA: its 128 rows of the
+//             two 256-row halves (two accumulators).
+// The leader CTA (rank 0) issues the MMAs; loads of both CTAs complete on the
+// leader's stage barrier (cta_group::2 tensor loads, no multicast); the
+// leader's commits arrive on the barrier at the same offset in both CTAs.
+// The second CTA's gathered token rows (cp.async) complete on its own barrier
+// and are forwarded to the leader by its otherwise idle MMA warp.
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
+    moe_gemm_pair_kernel(const __grid_constant__ GemmParams p) {
+  static_assert(MODE == kModeGateUp || MODE == kModeDown, "pair kernel serves the expert GEMMs");
+  // gate/up: gate and up tile of this CTA's 128 rows; down: one 128-row tile.
+  constexpr int NA = (MODE == kModeGateUp) ? 2 : 1;
+  constexpr int EW = epi_warps_of(MODE);
+  constexpr int kWbRows = 2 * kTileRows;   // weight rows per pair-unit (128 per CTA)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + (kSmemAlign - 1)) & ~static_cast<uintptr_t>(kSmemAlign - 1));
+  const int nmax = p.nmax;
+  const int S = p.stages;
+  const uint32_t stage_bytes = NA * kATileBytes + static_cast<uint32_t>(nmax / 2) * 128u;
+  uint8_t* epi = smem + static_cast<size_t>(S) * stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi + kEpiBytes);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + kMaxTmemBufs;
+  uint64_t* drain = tempty + kMaxTmemBufs;
+  uint64_t* gfull = drain + 1;                       // rank 1, gate/up: its own gathers landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gfull + S);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      // leader: both producers' expect-tx arrivals (+ gate/up: its 128 gathering
+      // threads and the forwarded arrival of the second CTA's gathers)
+      mbar_init(full + s, MODE == kModeGateUp ? 2 + kGatherThreads + 1 : 2);
+      mbar_init(empty + s, 1);
+      mbar_init(gfull + s, kGatherThreads);
+    }
+    for (int b = 0; b < kMaxTmemBufs; ++b) {
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, 2 * EW);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < 4; ++i) prefetch_tensormap(&p.mapA[i]);
+    if (MODE == kModeDown)
+      for (int i = 0; i < 4; ++i) prefetch_tensormap(&p.mapB[0][i]);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                    // peer barriers are initialised
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_units = *p.num_units_dev;
+  const uint32_t full_leader = mapa_shared(smem_u32(full), 0);     // + 8 * stage
+  const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0); // + 8 * buf
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ weight (and down: token) loads
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0;
+    bool ok = true;
+    for (int u = pair; ok && u < num_units; u += npairs) {
+      const Unit un = get_unit<MODE>(p, u);
+      const bool sh = un.g >= p.E;
+      const int sidx = sh ? un.g - p.E : 0;
+      const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
+      const int KB = K / kTileK;
+      const CUtensorMap* mA = &p.mapA[sh ? 2 : 0];
+      const CUtensorMap* mB = p.mapB[sh ? 1 : 0];
+      const int a_c2 = sh ? sidx : un.g;
+      const int half = un.n >> 1;
+      const int brow0 = (sh ? sidx * p.Tp : 0) + un.row0 + static_cast<int>(rank) * half;
+      const uint32_t tx_bytes = NA * kATileBytes + (MODE == kModeDown ? static_cast<uint32_t>(half) * 128u : 0u);
+      int got = 1;
+      if (lane == 0) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
+            got = 0;
+            break;
+          }
+          const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+          const uint32_t fb = full_leader + 8u * stage;
+          mbar_arrive_expect_tx_cluster(fb, tx_bytes);
+#pragma unroll
+          for (int a = 0; a < NA; ++a)
+            tma_load_3d_pair(sbase + a * kATileBytes, mA + a, fb, kb * kTileK,
+                             un.wb * kWbRows + static_cast<int>(rank) * kTileRows, a_c2);
+          if (MODE == kModeDown)
+            tma_load_rows<true>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, half);
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) ok = false;
+    }
+    // The leader's stage barriers count both CTAs' bytes: drain the last ones.
+    if (lane == 0 && rank == 0) {
+      const uint32_t outstanding = issued < static_cast<uint32_t>(S) ? issued : static_cast<uint32_t>(S);
+      for (uint32_t i = 1; i <= outstanding; ++i) {
+        const uint32_t I = issued - i;
+        mbar_wait_drain(&full[I % S], (I / S) & 1u, p.timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------------- MMA issuer (leader)
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t ucount = 0;
+      bool any = false;
+      bool ok = true;
+      for (int u = pair; ok && u < num_units; u += npairs) {
+        const Unit un = get_unit<MODE>(p, u);
+        const bool sh = un.g >= p.E;
+        const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
+        const int KB = K / kTileK;
+        const int buf = static_cast<int>(ucount % static_cast<uint32_t>(p.nbuf));
+        const uint32_t bpar = (ucount / static_cast<uint32_t>(p.nbuf)) & 1u;
+        if (!mbar_wait(&tempty[buf], bpar ^ 1u, abort_flag, p.err, p.timeout_ns)) break;
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16_f32(2 * kTileRows, un.n);
+        const uint32_t dcol = tmem_base + static_cast<uint32_t>(buf * NA * nmax);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (MODE == kModeGateUp) fence_proxy_async_smem();
+          const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+          const uint64_t bdesc = sw128_kmajor_desc(sbase + NA * kATileBytes);
+          uint64_t adesc[NA];
+#pragma unroll
+          for (int a = 0; a < NA; ++a) adesc[a] = sw128_kmajor_desc(sbase + a * kATileBytes);
+#pragma unroll
+          for (int ks = 0; ks < kTileK / 16; ++ks) {
+#pragma unroll
+            for (int a = 0; a < NA; ++a)
+              tc_mma_bf16_pair(dcol + static_cast<uint32_t>(a * nmax), adesc[a] + 2u * ks, bdesc + 2u * ks, idesc,
+                               (kb | ks) != 0 ? 1u : 0u);
+          }
+          any = true;
+          tc_commit_pair(&empty[stage], 0x3);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(&tfull[buf], 0x3);
+        ++ucount;
+      }
+      if (any) {
+        tc_commit_pair(drain, 0x1);
+        mbar_wait_drain(drain, 0, p.timeout_ns);
+      }
+    } else if (lane == 0 && MODE == kModeGateUp) {
+      // ---------------------------------------------------------- rank 1: forward gather completion
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = pair; ok && u < num_units; u += npairs) {
+        const int KB = p.d / kTileK;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&gfull[stage], phase, abort_flag, p.err, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive_cluster(full_leader + 8u * stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (MODE == kModeGateUp && warp >= 2 + EW) {
+    // ------------------------------------------------------------ row gather (this CTA's half)
+    const int g = threadIdx.x - 32 * (2 + EW);
+    const int part = g & 7;
+    const int r0 = g >> 3;
+    uint64_t* land = (rank == 0) ? full : gfull;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int u = pair; ok && u < num_units; u += npairs) {
+      const Unit un = get_unit<MODE>(p, u);
+      const bool sh = un.g >= p.E;
+      const int half = un.n >> 1;
+      const int nr = (r0 < half) ? (half - r0 + 15) >> 4 : 0;      // rows r0 + 16 i < half
+      const int rbase = un.row0 + static_cast<int>(rank) * half;
+      int tok[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = rbase + r0 + 16 * i;
+        tok[i] = (i < nr) ? min(max(sh ? r : __ldg(p.perm + r), 0), p.T - 1) : 0;
+      }
+      const int KB = p.d / kTileK;
+      for (int kb = 0; kb < KB; ++kb) {
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          ok = false;
+          break;
+        }
+        const uint32_t bbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + NA * kATileBytes;
+        const __nv_bfloat16* src0 = reinterpret_cast<const __nv_bfloat16*>(p.x) + kb * kTileK + part * 8;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (i < nr) {
+            const int r = r0 + 16 * i;
+            cp_async_16(bbase + r * 128 + ((part ^ (r & 7)) << 4), src0 + static_cast<size_t>(tok[i]) * p.d);
+          }
+        }
+        cp_async_mbar_arrive_noinc(&land[stage]);
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    cp_async_wait_all();
+  } else if (warp >= 2 && warp < 2 + EW) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    uint8_t* stg = epi + (warp - 2) * (kEpiBytes / EW);
+    uint32_t ucount = 0;
+    for (int u = pair; u < num_units; u += npairs) {
+      const Unit un = get_unit<MODE>(p, u);
+      const bool sh = un.g >= p.E;
+      const int sidx = sh ? un.g - p.E : 0;
+      const int buf = static_cast<int>(ucount % static_cast<uint32_t>(p.nbuf));
+      const uint32_t bpar = (ucount / static_cast<uint32_t>(p.nbuf)) & 1u;
+      // down: combine weights of the unit's rows, fetched before the wait
+      // (lane l of register j holds the weight of column 32 j + l)
+      float wreg[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = 32 * j + lane;
+        wreg[j] = (MODE == kModeDown && !sh && c < un.n) ? __ldg(p.roww + un.row0 + c) : 1.0f;
+      }
+      int got = 1;
+      if (lane == 0) got = mbar_wait(&tfull[buf], bpar, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) break;
+      tc_fence_after();
+      const int half = (warp - 2) >> 2;                                   // column blocks half*16 + 32 i
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * NA * nmax);
+      const int feat0 = un.wb * kWbRows + static_cast<int>(rank) * kTileRows + 32 * q;
+      const int wrows = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
+      if (feat0 < wrows) {
+        const int ld = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
+        __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(sh ? p.out_s : p.out_r);
+        const size_t rbase = (sh ? static_cast<size_t>(sidx) * p.Tp : 0) + static_cast<size_t>(un.row0);
+        auto emit = [&](const uint32_t (&A)[16], const uint32_t (&B)[16], int c, float wsel) {
+          __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
+          if (MODE == kModeGateUp) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float gg = __uint_as_float(A[i]);
+              const float vv = __uint_as_float(B[i]);
+              sb[i * 32 + lane] = __float2bfloat16_rn(silu_f(gg) * vv);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float w = __shfl_sync(0xffffffffu, wsel, (c + i) & 31);
+              sb[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(A[i]) * w);
+            }
+          }
+          __syncwarp();
+#pragma unroll
+          for (int rep = 0; rep < 2; ++rep) {
+            const int cc = lane + 32 * rep;
+            const int tok = cc >> 2, part = cc & 3;
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + tok * 64 + part * 16);
+            *reinterpret_cast<uint4*>(outp + (rbase + c + tok) * ld + feat0 + part * 8) = v;
+          }
+          __syncwarp();
+        };
+        constexpr int kStep = 32;
+        uint32_t a0[16], b0[16], a1[16], b1[16];
+        int c0 = 16 * half;
+        if (c0 < un.n) {
+          tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c0), a0);
+          if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c0), b0);
+        }
+        while (c0 < un.n) {
+          tmem_ld_wait();
+          const int c1 = c0 + kStep;
+          if (c1 < un.n) {
+            tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c1), a1);
+            if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c1), b1);
+          }
+          emit(a0, b0, c0, MODE == kModeDown ? pick8(wreg, c0 >> 5) : 1.0f);
+          if (c1 >= un.n) break;
+          tmem_ld_wait();
+          const int c2 = c1 + kStep;
+          if (c2 < un.n) {
+            tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c2), a0);
+            if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c2), b0);
+          }
+          emit(a1, b1, c1, MODE == kModeDown ? pick8(wreg, c1 >> 5) : 1.0f);
+          c0 = c2;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + 8u * buf);
+      ++ucount;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                    // no CTA leaves while its peer may still touch it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 }  // namespace
 
 size_t gemm_smem_bytes(int mode, int nmax, int* stages) {
@@ -540,6 +909,43 @@ size_t gemm_smem_bytes(int mode, int nmax, int* stages) {
   if (s > kMaxStages) s = kMaxStages;
   if (stages) *stages = s;
   return fixed + static_cast<size_t>(s) * stage_bytes;
+}
+
+size_t gemm_pair_smem_bytes(int mode, int nmax, int* stages) {
+  const int NA = (mode == kModeGateUp) ? 2 : 1;
+  const size_t stage_bytes = NA * static_cast<size_t>(kATileBytes) + static_cast<size_t>(nmax / 2) * 128;
+  const size_t fixed = kSmemAlign + kEpiBytes + kSmemTail;
+  const size_t budget = 232448;
+  int s = static_cast<int>((budget - fixed) / stage_bytes);
+  if (s > kMaxStages) s = kMaxStages;
+  if (stages) *stages = s;
+  return fixed + static_cast<size_t>(s) * stage_bytes;
+}
+
+template <int MODE>
+static int launch_pair_mode(const GemmParams& prm, int grid, size_t smem, cudaStream_t st) {
+  static int configured[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  if (configured[dev] < static_cast<int>(smem)) {
+    if (cudaFuncSetAttribute(moe_gemm_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured[dev] = static_cast<int>(smem);
+  }
+  moe_gemm_pair_kernel<MODE><<<grid, threads_of(MODE), smem, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_gemm_pair(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st) {
+  grid &= ~1;
+  if (grid < 2) return MOE_ERR_UNSUPPORTED;
+  switch (mode) {
+    case kModeGateUp: return launch_pair_mode<kModeGateUp>(prm, grid, smem, st);
+    case kModeDown: return launch_pair_mode<kModeDown>(prm, grid, smem, st);
+    default: return MOE_ERR_INVALID_ARG;
+  }
 }
 
 template <int MODE>

@@ -26,16 +26,19 @@ struct Plan {
   // shape
   int T, d, E, k, f, S, fs;
   // derived sizes
-  int Tp;          // T rounded up to kRowPad
-  int Rcap;        // routed row capacity: T*k + E*(kRowPad-1), rounded to kRowPad
+  int pair1;       // 1: the gate/up GEMM runs on CTA pairs (cta_group::2)
+  int pair2;       // 1: the down GEMM runs on CTA pairs
+  int rowpad;      // expert segments (and T) are padded to this many rows: 32 with pairs, else 16
+  int Tp;          // T rounded up to rowpad
+  int Rcap;        // routed row capacity: T*k + E*(rowpad-1), rounded to rowpad
   int nb;          // permute blocks: ceil(T / kPermBlock)
   int nmax_r;      // tokens per router work unit
   int nmax1;       // rows per gate/up work unit (MMA N max)
   int nmax2;       // rows per down work unit
   int nwbE;        // 128-row blocks of E
-  int nwb1;        // 128-row blocks of f
-  int nwb1s;       // 128-row blocks of fs
-  int nwb2;        // 256-row blocks of d (down-projection units)
+  int nwb1;        // weight blocks of f per gate/up unit: 128 rows (256 with pairs)
+  int nwb1s;       // the same for fs
+  int nwb2;        // weight blocks of d per down unit: 256 rows
   int router_units;
   int U1cap, U2cap;
   int shared_units1, shared_units2;
@@ -61,7 +64,7 @@ enum GemmMode { kModeRouter = 0, kModeGateUp = 1, kModeDown = 2 };
 
 struct GemmParams {
   CUtensorMap mapA[4];      // A operands: [0],[1] routed (gate, up | down | router); [2],[3] shared
-  CUtensorMap mapB[2];      // B sources: [0] routed / all tokens, [1] shared (down only)
+  CUtensorMap mapB[2][4];   // token-row sources ([0] routed / all tokens, [1] shared), boxes of 16/32/64/128 rows
   const int4* units;        // work list (gate/up and down)
   const int* num_units_dev; // its length, on the device
   int num_units_host;       // router: number of units
@@ -78,6 +81,9 @@ struct GemmParams {
 
 int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st);
 size_t gemm_smem_bytes(int mode, int nmax, int* stages);
+// CTA-pair (cta_group::2) expert GEMMs; grid is rounded down to an even count.
+int launch_gemm_pair(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st);
+size_t gemm_pair_smem_bytes(int mode, int nmax, int* stages);
 
 int launch_topk(const float* logits, const float* bias, int T, int E, int k, int score_fn,
                 int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w,

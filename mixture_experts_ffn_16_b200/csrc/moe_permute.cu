@@ -13,10 +13,11 @@
 //             the lower warps and of its own warp: rows inside an expert are in
 //             ascending token order, so the layout is deterministic.
 //
-// Row space: expert e owns rows [roff[e], roff[e] + pad16(count[e])); padding
+// Row space: expert e owns rows [roff[e], roff[e] + pad(count[e])) with
+// pad() rounding up to 16 rows (32 when the expert GEMMs run on CTA pairs); padding
 // rows point at token 0 with weight 0.  Work units are int4
-// {group, 128-row weight block, first row, rows (multiple of 16)}; shared
-// experts are groups E..E+S-1 over rows 0..pad16(T) of their own row space and
+// {group, weight block, first row, rows (a multiple of the padding)}; shared
+// experts are groups E..E+S-1 over rows 0..pad(T) of their own row space and
 // come first in each list.
 #include "moe_internal.h"
 #include "moe_ptx.cuh"
@@ -96,7 +97,7 @@ struct ScanArgs {
   int4* units1;
   int4* units2;
   int32_t* nunits;   // [4]: gate/up units, down units, padded routed rows, 0
-  int nb, E, T, Tp;
+  int nb, E, T, Tp, rowpad;
   int nmax1, nmax2, nwb1, nwb1s, nwb2, S;
   int shared_units1, shared_units2;
 };
@@ -112,16 +113,23 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) 
     const int e = threadIdx.x * kPer + i;
     int c = 0;
     if (e < a.E) {
-      for (int b = 0; b < a.nb; ++b) {
-        int32_t* p = a.blkcnt + static_cast<size_t>(b) * a.E + e;
-        const int v = *p;
-        *p = c;
-        c += v;
+      // Column e of the block histogram: exclusive prefix over blocks.  The
+      // loads of a batch are issued before any store so they overlap.
+      int32_t* col = a.blkcnt + e;
+      for (int b0 = 0; b0 < a.nb; b0 += 16) {
+        int v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = (b0 + j < a.nb) ? col[static_cast<size_t>(b0 + j) * a.E] : 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if (b0 + j < a.nb) col[static_cast<size_t>(b0 + j) * a.E] = c;
+          c += v[j];
+        }
       }
       a.counts[e] = c;
     }
     cnt[i] = c;
-    pad[i] = (c + kRowPad - 1) / kRowPad * kRowPad;
+    pad[i] = (c + a.rowpad - 1) / a.rowpad * a.rowpad;
     u1[i] = (pad[i] + a.nmax1 - 1) / a.nmax1 * a.nwb1;
     u2[i] = (pad[i] + a.nmax2 - 1) / a.nmax2 * a.nwb2;
     sp += pad[i];
@@ -238,6 +246,7 @@ int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, 
   a.E = p.E;
   a.T = p.T;
   a.Tp = p.Tp;
+  a.rowpad = p.rowpad;
   a.nmax1 = p.nmax1;
   a.nmax2 = p.nmax2;
   a.nwb1 = p.nwb1;

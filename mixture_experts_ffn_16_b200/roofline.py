@@ -9,6 +9,7 @@ Counts only what the method must do, not what an implementation moves:
 """
 from __future__ import annotations
 
+import hashlib
 import json
 import os
 
@@ -62,3 +63,31 @@ def block_cost(cfg, touched=None):
     flops = 2.0 * T * E * d + 2.0 * T * k * 3 * f * d + 2.0 * T * S * 3 * fs * d
     bytes_ = 2.0 * (ne * 3 * f * d + S * 3 * fs * d + E * d + 2 * T * d) + 8.0 * T * k
     return flops, bytes_
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch, from
+# the ncu captures summarised in profiles/gemm_<workload>.md.  A figure is
+# valid only while the GEMM source is the one that was captured (sha256 prefix).
+NCU_TRAFFIC = {
+    ("prefill_softmax", "route"): (17.9e6, "9086017a9f5ca9dc"),
+    ("prefill_softmax", "gate_up"): (1209.6e6, "9086017a9f5ca9dc"),
+    ("prefill_softmax", "down"): (719.3e6, "9086017a9f5ca9dc"),
+}
+
+
+def _gemm_source_sha():
+    p = os.path.join(ROOT, "mixture_experts_ffn_16_b200", "csrc", "moe_gemm.cu")
+    try:
+        with open(p, "rb") as fh:
+            return hashlib.sha256(fh.read()).hexdigest()[:16]
+    except OSError:
+        return None
+
+
+def measured_traffic(workload, kernel):
+    """Bytes per launch from the committed capture, or None when there is none
+    or the kernel source has changed since it was taken."""
+    rec = NCU_TRAFFIC.get((workload, kernel))
+    if rec is None or _gemm_source_sha() != rec[1]:
+        return None
+    return rec[0]
