@@ -146,6 +146,7 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* 
   g.T = p.T; g.Tp = p.Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
   g.nmax = p.nmax1;
   g.timeout_ns = kWaitTimeoutNs;
+  g.weights_evict_first = p.weights_evict_first;
   int stages = 0;
   g.nbuf = (2 * p.nmax1 <= 256) ? 2 : 1;
   if (p.pair1) {
@@ -181,6 +182,7 @@ int run_down(const Plan& p, const DeviceInfo& di, const void* Wd, const void* Ws
   g.T = p.T; g.Tp = p.Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
   g.nmax = p.nmax2;
   g.timeout_ns = kWaitTimeoutNs;
+  g.weights_evict_first = p.weights_evict_first;
   int stages = 0;
   if (p.pair2) {
     g.nbuf = (p.nmax2 <= 256) ? 2 : 1;          // one accumulator per CTA
@@ -254,6 +256,8 @@ int make_plan(const moe_shape* s, Plan* p) {
   q.pair1 = (q.nmax1 >= 64 && rows_per_expert >= 256.0) ? 1 : 0;
   q.pair2 = 0;
   q.rowpad = (q.pair1 || q.pair2) ? 2 * kRowPad : kRowPad;
+  // Experts that fit one token run on average read each weight tile once.
+  q.weights_evict_first = rows_per_expert <= 0.75 * q.nmax1 ? 1 : 0;
   q.Tp = ceil_div(T, q.rowpad) * q.rowpad;
   q.Rcap = ceil_div(T * k + E * (q.rowpad - 1), q.rowpad) * q.rowpad;
   q.nb = ceil_div(T, kPermBlock);
@@ -263,13 +267,18 @@ int make_plan(const moe_shape* s, Plan* p) {
   q.nwb1 = ceil_div(f, rows1);
   q.nwb1s = S > 0 ? ceil_div(fs, rows1) : 0;
   q.nwb2 = ceil_div(d, rows2);
-  // Router: runs of up to 64 tokens (their fp32 logit sums live in registers);
-  // narrower runs only when that leaves most SMs of a B200 idle.
+  // Router: runs of up to 128 tokens (their fp32 logit sums live in
+  // registers) when that still gives every SM of a B200 a unit; else runs of
+  // 64 or narrower while most SMs stay busy.
   q.nmax_r = 16;
-  for (int n = 64; n >= 16; n >>= 1) {
-    if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, n) >= 74) {
-      q.nmax_r = n;
-      break;
+  if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, 128) >= 148) {
+    q.nmax_r = 128;
+  } else {
+    for (int n = 64; n >= 16; n >>= 1) {
+      if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, n) >= 74) {
+        q.nmax_r = n;
+        break;
+      }
     }
   }
   q.router_units = q.nwbE * ceil_div(q.Tp, q.nmax_r);

@@ -49,7 +49,7 @@ constexpr int kSmemAlign = 1024;
 constexpr int kSmemTail = 512;                       // barriers, TMEM slot, abort flag
 constexpr int kMaxTmemBufs = 8;                      // accumulator buffers (router: 8 x 64 columns)
 constexpr int kRouterDrainKB = 2;                    // router: k-blocks accumulated in TMEM per drain
-constexpr int kRouterMaxN = 64;                      // router: tokens per unit (fp32 sums in registers)
+constexpr int kRouterMaxN = 128;                     // router: tokens per unit (fp32 sums in registers)
 
 struct Unit {
   int g, wb, row0, n;
@@ -152,6 +152,12 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // router: W_router and x are re-read by every unit -> keep; expert
+    // weights that stream through once -> evict first; expert weights that
+    // several token runs of one expert share -> keep.
+    const uint64_t pol_a = (MODE == kModeRouter || !p.weights_evict_first) ? policy_evict_last()
+                                                                           : policy_evict_first();
+    const uint64_t pol_b = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued = 0;
@@ -182,10 +188,10 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
           mbar_arrive_expect_tx(&full[stage], tx_bytes);
 #pragma unroll
           for (int a = 0; a < NA; ++a)
-            tma_load_3d(sbase + a * kATileBytes, (MODE == kModeDown) ? mA : mA + a, fb, kb * kTileK,
-                        un.wb * kWbRows + ((MODE == kModeDown) ? a * kTileRows : 0), a_c2);
+            tma_load_3d_hint(sbase + a * kATileBytes, (MODE == kModeDown) ? mA : mA + a, fb, kb * kTileK,
+                             un.wb * kWbRows + ((MODE == kModeDown) ? a * kTileRows : 0), a_c2, pol_a);
           if (MODE != kModeGateUp)
-            tma_load_rows<false>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, un.n);
+            tma_load_rows<false>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, un.n, pol_b);
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -317,6 +323,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
     const int g = threadIdx.x - 32 * (2 + epi_warps_of(MODE));
     const int part = g & 7;
     const int r0 = g >> 3;
+    const uint64_t pol_x = policy_evict_last();     // x rows are gathered by every weight block
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -346,7 +353,8 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
         for (int i = 0; i < 16; ++i) {
           if (i < nr) {
             const int r = r0 + 16 * i;
-            cp_async_16(bbase + r * 128 + ((part ^ (r & 7)) << 4), src0 + static_cast<size_t>(tok[i]) * p.d);
+            cp_async_16(bbase + r * 128 + ((part ^ (r & 7)) << 4), src0 + static_cast<size_t>(tok[i]) * p.d,
+                        pol_x);
           }
         }
         cp_async_mbar_arrive_noinc(&full[stage]);
@@ -389,14 +397,22 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
           if (live) {
             const uint32_t tb =
                 tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * nmax);
-            uint32_t v[4][16];
+            // 64 columns per round trip: 4 loads in flight, then add.
 #pragma unroll
-            for (int c = 0; c < kRouterMaxN / 16; ++c) tmem_ld_32x32b_x16(tb + 16u * c, v[c]);
-            tmem_ld_wait();
+            for (int g = 0; g < kRouterMaxN / 64; ++g) {
+              if (64 * g < un.n) {
+                uint32_t v[4][16];
 #pragma unroll
-            for (int c = 0; c < kRouterMaxN / 16; ++c)
+                for (int c = 0; c < 4; ++c)
+                  if (64 * g + 16 * c < un.n) tmem_ld_32x32b_x16(tb + static_cast<uint32_t>(64 * g + 16 * c), v[c]);
+                tmem_ld_wait();
 #pragma unroll
-              for (int j = 0; j < 16; ++j) acc[16 * c + j] += __uint_as_float(v[c][j]);
+                for (int c = 0; c < 4; ++c)
+                  if (64 * g + 16 * c < un.n)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) acc[64 * g + 16 * c + j] += __uint_as_float(v[c][j]);
+              }
+            }
           }
           tc_fence_before();
           __syncwarp();
@@ -625,6 +641,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ weight (and down: token) loads
+    const uint64_t pol_a = p.weights_evict_first ? policy_evict_first() : policy_evict_last();
+    const uint64_t pol_b = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued = 0;
@@ -653,10 +671,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
           mbar_arrive_expect_tx_cluster(fb, tx_bytes);
 #pragma unroll
           for (int a = 0; a < NA; ++a)
-            tma_load_3d_pair(sbase + a * kATileBytes, mA + a, fb, kb * kTileK,
-                             un.wb * kWbRows + static_cast<int>(rank) * kTileRows, a_c2);
+            tma_load_3d_pair_hint(sbase + a * kATileBytes, mA + a, fb, kb * kTileK,
+                                  un.wb * kWbRows + static_cast<int>(rank) * kTileRows, a_c2, pol_a);
           if (MODE == kModeDown)
-            tma_load_rows<true>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, half);
+            tma_load_rows<true>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, half, pol_b);
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -756,6 +774,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
     const int part = g & 7;
     const int r0 = g >> 3;
     uint64_t* land = (rank == 0) ? full : gfull;
+    const uint64_t pol_x = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -786,7 +805,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
         for (int i = 0; i < 8; ++i) {
           if (i < nr) {
             const int r = r0 + 16 * i;
-            cp_async_16(bbase + r * 128 + ((part ^ (r & 7)) << 4), src0 + static_cast<size_t>(tok[i]) * p.d);
+            cp_async_16(bbase + r * 128 + ((part ^ (r & 7)) << 4), src0 + static_cast<size_t>(tok[i]) * p.d,
+                        pol_x);
           }
         }
         cp_async_mbar_arrive_noinc(&land[stage]);

@@ -29,6 +29,7 @@ struct Plan {
   int pair1;       // 1: the gate/up GEMM runs on CTA pairs (cta_group::2)
   int pair2;       // 1: the down GEMM runs on CTA pairs
   int rowpad;      // expert segments (and T) are padded to this many rows: 32 with pairs, else 16
+  int weights_evict_first;  // expert weight tiles are read once per call (L2 evict-first)
   int Tp;          // T rounded up to rowpad
   int Rcap;        // routed row capacity: T*k + E*(rowpad-1), rounded to rowpad
   int nb;          // permute blocks: ceil(T / kPermBlock)
@@ -77,6 +78,7 @@ struct GemmParams {
   int T, Tp, E, d, f, fs;
   int nmax, stages, nbuf, router_nwb;
   uint64_t timeout_ns;
+  int weights_evict_first;  // 1: each weight tile is read by one unit (experts fit one token run)
 };
 
 int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st);

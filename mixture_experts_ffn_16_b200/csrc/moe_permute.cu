@@ -71,21 +71,44 @@ permute_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
   }
 }
 
-// Exclusive block-wide scan of one int per thread (kScanThreads threads).
-__device__ int block_exclusive_scan(int v, int* sh, int* total) {
-  const int tid = threadIdx.x;
-  sh[tid] = v;
-  __syncthreads();
-  for (int off = 1; off < kScanThreads; off <<= 1) {
-    const int add = tid >= off ? sh[tid - off] : 0;
-    __syncthreads();
-    sh[tid] += add;
-    __syncthreads();
+// Exclusive block-wide scan of three ints per thread (kScanThreads threads):
+// shuffles inside each warp, then one warp scans the 32 warp totals.
+__device__ int3 block_exclusive_scan3(int3 v, int3* total) {
+  __shared__ int3 wsum[kScanThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int3 inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, inc.x, o);
+    const int y = __shfl_up_sync(0xffffffffu, inc.y, o);
+    const int z = __shfl_up_sync(0xffffffffu, inc.z, o);
+    if (lane >= o) {
+      inc.x += x;
+      inc.y += y;
+      inc.z += z;
+    }
   }
-  const int incl = sh[tid];
-  *total = sh[kScanThreads - 1];
+  if (lane == 31) wsum[warp] = inc;
   __syncthreads();
-  return incl - v;
+  if (warp == 0) {
+    int3 w = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, w.x, o);
+      const int y = __shfl_up_sync(0xffffffffu, w.y, o);
+      const int z = __shfl_up_sync(0xffffffffu, w.z, o);
+      if (lane >= o) {
+        w.x += x;
+        w.y += y;
+        w.z += z;
+      }
+    }
+    wsum[lane] = w;                              // inclusive over warps
+  }
+  __syncthreads();
+  const int3 base = warp > 0 ? wsum[warp - 1] : make_int3(0, 0, 0);
+  *total = wsum[kScanThreads / 32 - 1];
+  return make_int3(base.x + inc.x - v.x, base.y + inc.y - v.y, base.z + inc.z - v.z);
 }
 
 struct ScanArgs {
@@ -103,7 +126,6 @@ struct ScanArgs {
 };
 
 __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) {
-  __shared__ int sh[kScanThreads];
   // Experts per thread: E <= 2048 -> at most 2.
   constexpr int kPer = (kMaxE + kScanThreads - 1) / kScanThreads;
   int cnt[kPer], pad[kPer], u1[kPer], u2[kPer];
@@ -136,10 +158,12 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) 
     s1 += u1[i];
     s2 += u2[i];
   }
-  int tot_rows, tot1, tot2;
-  int ro = block_exclusive_scan(sp, sh, &tot_rows);
-  int o1 = a.shared_units1 + block_exclusive_scan(s1, sh, &tot1);
-  int o2 = a.shared_units2 + block_exclusive_scan(s2, sh, &tot2);
+  int3 tot;
+  const int3 ex = block_exclusive_scan3(make_int3(sp, s1, s2), &tot);
+  const int tot_rows = tot.x, tot1 = tot.y, tot2 = tot.z;
+  int ro = ex.x;
+  int o1 = a.shared_units1 + ex.y;
+  int o2 = a.shared_units2 + ex.z;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = threadIdx.x * kPer + i;
