@@ -16,6 +16,7 @@ bounded sample of the same workload on rank 0; other ranks exit at once.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -39,6 +40,7 @@ from mixture_experts_ffn_16_b200.roofline import (block_cost, kernel_costs, meas
 METRIC = "MoE-layer tokens/sec at 1 B200; % bf16 tensor peak (prefill) / % HBM BW (decode)"
 STAGES = ["route", "permute", "gate_up", "down", "combine"]
 LAUNCHES_PER_STEP = {"route": 2, "permute": 3, "gate_up": 1, "down": 1, "combine": 1}
+SHARED_GATE_LAUNCHES = 1      # the per-token shared-expert gate kernel
 REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
@@ -55,6 +57,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--variant", default="", choices=["", "gated_shared", "external_routing"],
+                    help="gated_shared: Qwen3.5-style sigmoid gate on the shared experts; "
+                         "external_routing: routing supplied by the caller (steps a3..a7 only)")
     return ap.parse_args()
 
 
@@ -226,15 +231,24 @@ def run_ours(args, cfg):
     stream = torch.cuda.current_stream(dev)
     s = layer.shape
 
+    external = args.variant == "external_routing"
+    if external:
+        # the caller's routing: computed once, outside the timed steps
+        ext_idx, ext_w = layer.topk_idx.clone(), layer.topk_w.clone()
+        api.moe_route(s, inp["x"], inp["W_router"], inp["expert_bias"], cfg.score_fn, cfg.norm_topk,
+                      cfg.route_scale, ext_idx, ext_w, layer.workspace, stream)
+
     def step(ev=None):
         t, c = inp, cfg
         if ev is not None:
             ev[0].record(stream)
-        api.moe_route(s, t["x"], t["W_router"], t["expert_bias"], c.score_fn, c.norm_topk, c.route_scale,
-                      layer.topk_idx, layer.topk_w, layer.workspace, stream)
+        if not external:
+            api.moe_route(s, t["x"], t["W_router"], t["expert_bias"], c.score_fn, c.norm_topk, c.route_scale,
+                          layer.topk_idx, layer.topk_w, layer.workspace, stream)
         if ev is not None:
             ev[1].record(stream)
-        api.moe_permute(s, layer.topk_idx, layer.topk_w, layer.workspace, stream)
+        api.moe_permute(s, ext_idx if external else layer.topk_idx, ext_w if external else layer.topk_w,
+                        layer.workspace, stream)
         if ev is not None:
             ev[2].record(stream)
         api.moe_expert_gate_up(s, t["x"], t["W_gate"], t["W_up"], t["W_shared_gate"], t["W_shared_up"],
@@ -244,7 +258,8 @@ def run_ours(args, cfg):
         api.moe_expert_down(s, t["W_down"], t["W_shared_down"], layer.workspace, stream)
         if ev is not None:
             ev[4].record(stream)
-        api.moe_combine(s, layer.out, layer.workspace, stream)
+        api.moe_combine(s, layer.out, layer.workspace, stream, x=t["x"],
+                        W_shared_gate_vec=t.get("W_shared_gate_vec"))
         if ev is not None:
             ev[5].record(stream)
 
@@ -254,7 +269,7 @@ def run_ours(args, cfg):
     st = api.moe_device_status(layer.workspace, stream)
     if st != api.MOE_OK:
         raise RuntimeError(f"device status after warm-up: {api.status_string(st)}")
-    idx_host = layer.topk_idx.cpu().numpy()
+    idx_host = (ext_idx if external else layer.topk_idx).cpu().numpy()
     touched = int((np.bincount(idx_host.ravel(), minlength=cfg.E) > 0).sum())
 
     K = args.steps
@@ -278,7 +293,7 @@ def run_ours(args, cfg):
         raise RuntimeError(f"device status after timing: {api.status_string(st)}")
 
     # End to end through the public host-buffer entry point.  Like a server
-    # that feeds successive batches, the steps alternate between two streams,
+    # that feeds successive batches, the steps rotate over three streams,
     # each with its own workspace and page-locked buffers, so one batch's
     # host<->device copies overlap the other batch's kernels.  Every step
     # still copies its x in and its out / topk_idx / topk_w back inside the
@@ -286,7 +301,8 @@ def run_ours(args, cfg):
     e2e = None
     if not args.no_e2e:
         lanes = []
-        for li in range(2):
+        NL = 3
+        for li in range(NL):
             st_l = stream if li == 0 else torch.cuda.Stream(dev)
             lanes.append(dict(
                 stream=st_l,
@@ -297,12 +313,12 @@ def run_ours(args, cfg):
                 wh=torch.empty((cfg.T, cfg.k), dtype=torch.float32).pin_memory()))
 
         def host_step(i):
-            L = lanes[i % 2]
+            L = lanes[i % NL]
             api.moe_forward_host(s, L["xh"], inp["W_router"], inp["expert_bias"], inp["W_gate"], inp["W_up"],
                                  inp["W_down"], inp["W_shared_gate"], inp["W_shared_up"], inp["W_shared_down"],
                                  cfg.score_fn, cfg.norm_topk, cfg.route_scale, L["oh"], L["ih"], L["wh"], L["ws"],
-                                 L["stream"])
-        for i in range(max(4, args.warmup)):
+                                 L["stream"], W_shared_gate_vec=inp.get("W_shared_gate_vec"))
+        for i in range(max(2 * NL, args.warmup)):
             host_step(i)
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
@@ -310,7 +326,8 @@ def run_ours(args, cfg):
         barrier(world)
         torch.cuda.synchronize()
         e0.record(lanes[0]["stream"])
-        lanes[1]["stream"].wait_event(e0)
+        for L in lanes[1:]:
+            L["stream"].wait_event(e0)
         for i in range(K):
             host_step(i)
         for L, ev in zip(lanes, ends):
@@ -325,7 +342,7 @@ def run_ours(args, cfg):
         e2e = {"value": world * cfg.T * K / (e2e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": cfg.T * cfg.d * 2,
                "d2h_bytes_per_step": cfg.T * cfg.d * 2 + cfg.T * cfg.k * 8,
-               "streams": 2}
+               "streams": NL}
 
     value = world * cfg.T * K / (elapsed_ms / 1e3)
     peaks = measured_peaks()
@@ -367,12 +384,15 @@ def run_ours(args, cfg):
                 "config": {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "E": cfg.E, "k": cfg.k,
                            "d_ff": cfg.f, "n_shared": cfg.S, "d_ff_shared": cfg.fs, "score_fn": cfg.score_fn,
                            "norm_topk": cfg.norm_topk, "touched_experts": touched,
+                           "variant": args.variant or "base",
                            "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (
                                2.0 * cfg.E * 3 * cfg.f * cfg.d / 1e9),
                            "parallelism": "replicas" if world > 1 else "single GPU"},
                 "roofline": roof, "step_roofline": step_roof,
                 "kernels_us": stage_avg_us, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": K * sum(LAUNCHES_PER_STEP.values()),
+                "gpu_launches": K * (sum(LAUNCHES_PER_STEP.values())
+                                     - (LAUNCHES_PER_STEP["route"] if external else 0)
+                                     + (SHARED_GATE_LAUNCHES if cfg.shared_gate else 0)),
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -384,6 +404,8 @@ def run_ours(args, cfg):
 def main():
     args = parse()
     cfg = CONFIGS[args.config]
+    if args.variant == "gated_shared":
+        cfg = dataclasses.replace(cfg, shared_gate=True)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

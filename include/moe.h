@@ -99,6 +99,11 @@ MOE_API size_t moe_workspace_bytes(const moe_shape *shape);
 /* The whole block, steps a1..a7 below in order, on `stream`.
  *   x, weights: inputs as above.  expert_bias: fp32 [E] or NULL (selection
  *   only; ignored for MOE_SCORE_SOFTMAX).  W_shared_*: NULL iff S == 0.
+ *   W_shared_gate_vec: bf16 [S,d] or NULL.  NULL: shared experts are added
+ *   with weight 1 (DeepSeek-style).  Given: shared expert s is scaled per
+ *   token by sigmoid(W_shared_gate_vec[s] . x) before it is added (the
+ *   Qwen3.5 shared expert, qwen3-5-vs-gemma-4 component table, shared-expert
+ *   cell).  Requires S >= 1.
  *   score_fn: MOE_SCORE_*.  norm_topk: 0/1.  route_scale: multiplies the
  *   combine weights (1.0 = none; DeepSeek-V4-Pro uses 2.5).
  *   out      [T,d] bf16: the block output, residual-free.
@@ -110,6 +115,7 @@ MOE_API int moe_forward(const moe_shape *shape,
                 const void *x, const void *W_router, const float *expert_bias,
                 const void *W_gate, const void *W_up, const void *W_down,
                 const void *W_shared_gate, const void *W_shared_up, const void *W_shared_down,
+                const void *W_shared_gate_vec,
                 int score_fn, int norm_topk, float route_scale,
                 void *out, int32_t *topk_idx, float *topk_w,
                 void *workspace, size_t workspace_bytes, moe_stream_t stream);
@@ -124,6 +130,7 @@ MOE_API int moe_forward_host(const moe_shape *shape,
                      const void *x_host, const void *W_router, const float *expert_bias,
                      const void *W_gate, const void *W_up, const void *W_down,
                      const void *W_shared_gate, const void *W_shared_up, const void *W_shared_down,
+                     const void *W_shared_gate_vec,
                      int score_fn, int norm_topk, float route_scale,
                      void *out_host, int32_t *topk_idx_host, float *topk_w_host,
                      void *workspace, size_t workspace_bytes, moe_stream_t stream);
@@ -163,10 +170,27 @@ MOE_API int moe_expert_gate_up(const moe_shape *shape, const void *x,
 MOE_API int moe_expert_down(const moe_shape *shape, const void *W_down, const void *W_shared_down,
                     void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
-/* a7: out[t] = sum_s y_shared[s,t] + sum_{j<k} y[row(t,j)], summed in fp32 in
- * that fixed order and rounded to bf16 once (bitwise reproducible). */
-MOE_API int moe_combine(const moe_shape *shape, void *out,
+/* a7: out[t] = sum_s g[t,s] y_shared[s,t] + sum_{j<k} y[row(t,j)], summed in
+ * fp32 in that fixed order and rounded to bf16 once (bitwise reproducible).
+ * g = 1 when W_shared_gate_vec is NULL (x may then be NULL too), else
+ * sigmoid(W_shared_gate_vec[s] . x[t]) with x [T,d] the block input. */
+MOE_API int moe_combine(const moe_shape *shape, const void *x, const void *W_shared_gate_vec, void *out,
                 void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* External-indices mode: steps a3..a7 on a routing the caller supplies
+ * (for example experts picked by a fixed token-id hash, as the first MoE
+ * layers of DeepSeek-V4-Pro do, or an MTP layer reusing the trunk's routing:
+ * qwen3-5-vs-deepseek-v4 router cell; qwen3-5-vs-gemma-4 MTP cell).
+ *   topk_idx [T,k] int32: k distinct experts in [0,E) per token (violations
+ *   are reported by moe_device_status as MOE_ERR_INVALID_ARG; all indices
+ *   are clamped so nothing is read out of bounds).
+ *   topk_w [T,k] fp32: combine weights, used as given.
+ * Everything else as in moe_forward; clears the device error word. */
+MOE_API int moe_experts_forward(const moe_shape *shape, const void *x, const int32_t *topk_idx,
+                                const float *topk_w, const void *W_gate, const void *W_up,
+                                const void *W_down, const void *W_shared_gate, const void *W_shared_up,
+                                const void *W_shared_down, const void *W_shared_gate_vec, void *out,
+                                void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* Introspection of the workspace layout, for tests and debugging.  Regions:
  *   MOE_WS_LOGITS   fp32 [T,E]   router logits (after moe_route)

@@ -32,7 +32,7 @@ WS_REGIONS = {"logits": 0, "counts": 1, "offsets": 2, "perm": 3, "row_w": 4, "in
 EXPORTED = ["moe_version", "moe_status_string", "moe_workspace_bytes", "moe_forward",
             "moe_forward_host", "moe_route", "moe_permute", "moe_expert_gate_up", "moe_expert_down",
             "moe_combine", "moe_workspace_region", "moe_device_status", "moe_debug_wait_timeout",
-            "moe_route_noalloc"]
+            "moe_route_noalloc", "moe_experts_forward"]
 
 
 class MoEError(RuntimeError):
@@ -67,7 +67,7 @@ def load():
     lib.moe_status_string.argtypes = [I]
     lib.moe_workspace_bytes.restype = SZ
     lib.moe_workspace_bytes.argtypes = [SH]
-    fwd = [SH, P, P, P, P, P, P, P, P, P, I, I, ctypes.c_float, P, P, P, P, SZ, P]
+    fwd = [SH, P, P, P, P, P, P, P, P, P, P, I, I, ctypes.c_float, P, P, P, P, SZ, P]
     lib.moe_forward.restype = I
     lib.moe_forward.argtypes = fwd
     lib.moe_forward_host.restype = I
@@ -81,7 +81,9 @@ def load():
     lib.moe_expert_down.restype = I
     lib.moe_expert_down.argtypes = [SH, P, P, P, SZ, P]
     lib.moe_combine.restype = I
-    lib.moe_combine.argtypes = [SH, P, P, SZ, P]
+    lib.moe_combine.argtypes = [SH, P, P, P, P, SZ, P]
+    lib.moe_experts_forward.restype = I
+    lib.moe_experts_forward.argtypes = [SH, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.moe_workspace_region.restype = I
     lib.moe_workspace_region.argtypes = [SH, I, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]
     lib.moe_device_status.restype = I
@@ -179,16 +181,22 @@ def _weights(shape, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_d
             _p(W_shared_down, bf, (S, d, fs), "W_shared_down") if S else None]
 
 
+def _gate_vec(shape, W_shared_gate_vec):
+    if W_shared_gate_vec is None:
+        return None
+    return _p(W_shared_gate_vec, torch.bfloat16, (shape.n_shared, shape.d_model), "W_shared_gate_vec")
+
+
 def moe_forward(shape, x, W_router, expert_bias, W_gate, W_up, W_down, W_shared_gate, W_shared_up,
                 W_shared_down, score_fn, norm_topk, route_scale, out, topk_idx, topk_w, workspace,
-                stream=None):
+                stream=None, W_shared_gate_vec=None):
     T, d, E, k = shape.T, shape.d_model, shape.E, shape.k
     bf = torch.bfloat16
     st = load().moe_forward(
         ctypes.byref(shape), _p(x, bf, (T, d), "x"), _p(W_router, bf, (E, d), "W_router"),
         _p(expert_bias, torch.float32, (E,), "expert_bias"),
         *_weights(shape, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down),
-        _score(score_fn), int(bool(norm_topk)), float(route_scale),
+        _gate_vec(shape, W_shared_gate_vec), _score(score_fn), int(bool(norm_topk)), float(route_scale),
         _p(out, bf, (T, d), "out"), _p(topk_idx, torch.int32, (T, k), "topk_idx"),
         _p(topk_w, torch.float32, (T, k), "topk_w"),
         _p(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream))
@@ -197,14 +205,14 @@ def moe_forward(shape, x, W_router, expert_bias, W_gate, W_up, W_down, W_shared_
 
 def moe_forward_host(shape, x_host, W_router, expert_bias, W_gate, W_up, W_down, W_shared_gate,
                      W_shared_up, W_shared_down, score_fn, norm_topk, route_scale, out_host,
-                     topk_idx_host, topk_w_host, workspace, stream=None):
+                     topk_idx_host, topk_w_host, workspace, stream=None, W_shared_gate_vec=None):
     T, d, E, k = shape.T, shape.d_model, shape.E, shape.k
     bf = torch.bfloat16
     st = load().moe_forward_host(
         ctypes.byref(shape), _p(x_host, bf, (T, d), "x_host", host=True),
         _p(W_router, bf, (E, d), "W_router"), _p(expert_bias, torch.float32, (E,), "expert_bias"),
         *_weights(shape, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down),
-        _score(score_fn), int(bool(norm_topk)), float(route_scale),
+        _gate_vec(shape, W_shared_gate_vec), _score(score_fn), int(bool(norm_topk)), float(route_scale),
         _p(out_host, bf, (T, d), "out_host", host=True),
         _p(topk_idx_host, torch.int32, (T, k), "topk_idx_host", host=True),
         _p(topk_w_host, torch.float32, (T, k), "topk_w_host", host=True),
@@ -271,11 +279,27 @@ def moe_expert_down(shape, W_down, W_shared_down, workspace, stream=None):
     _check(st, "moe_expert_down")
 
 
-def moe_combine(shape, out, workspace, stream=None):
-    st = load().moe_combine(ctypes.byref(shape), _p(out, torch.bfloat16, (shape.T, shape.d_model), "out"),
+def moe_combine(shape, out, workspace, stream=None, x=None, W_shared_gate_vec=None):
+    T, d = shape.T, shape.d_model
+    st = load().moe_combine(ctypes.byref(shape), _p(x, torch.bfloat16, (T, d), "x"),
+                            _gate_vec(shape, W_shared_gate_vec), _p(out, torch.bfloat16, (T, d), "out"),
                             _p(workspace, torch.uint8, None, "workspace"), workspace.numel(),
                             _stream(stream))
     _check(st, "moe_combine")
+
+
+def moe_experts_forward(shape, x, topk_idx, topk_w, W_gate, W_up, W_down, W_shared_gate, W_shared_up,
+                        W_shared_down, out, workspace, stream=None, W_shared_gate_vec=None):
+    """Steps a3..a7 on a caller-supplied routing (external-indices mode)."""
+    T, d, k = shape.T, shape.d_model, shape.k
+    bf = torch.bfloat16
+    st = load().moe_experts_forward(
+        ctypes.byref(shape), _p(x, bf, (T, d), "x"), _p(topk_idx, torch.int32, (T, k), "topk_idx"),
+        _p(topk_w, torch.float32, (T, k), "topk_w"),
+        *_weights(shape, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down),
+        _gate_vec(shape, W_shared_gate_vec), _p(out, bf, (T, d), "out"),
+        _p(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "moe_experts_forward")
 
 
 def moe_device_status(workspace, stream=None) -> int:
@@ -318,7 +342,8 @@ class MoELayer:
         moe_forward(self.shape, t["x"] if x is None else x, t["W_router"], t["expert_bias"],
                     t["W_gate"], t["W_up"], t["W_down"], t["W_shared_gate"], t["W_shared_up"],
                     t["W_shared_down"], c.score_fn, c.norm_topk, c.route_scale, self.out,
-                    self.topk_idx, self.topk_w, self.workspace, stream)
+                    self.topk_idx, self.topk_w, self.workspace, stream,
+                    W_shared_gate_vec=t.get("W_shared_gate_vec"))
         return self.out, self.topk_idx, self.topk_w
 
     def steps(self, stream=None, events=None):
@@ -338,6 +363,6 @@ class MoELayer:
         rec(3)
         moe_expert_down(s, t["W_down"], t["W_shared_down"], self.workspace, st)
         rec(4)
-        moe_combine(s, self.out, self.workspace, st)
+        moe_combine(s, self.out, self.workspace, st, x=t["x"], W_shared_gate_vec=t.get("W_shared_gate_vec"))
         rec(5)
         return self.out, self.topk_idx, self.topk_w

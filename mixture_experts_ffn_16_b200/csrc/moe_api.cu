@@ -218,17 +218,34 @@ int check_expert_args(const Plan& p, const void* Wg, const void* Wu, const void*
   return MOE_OK;
 }
 
-int forward_impl(const Plan& p, const DeviceInfo& di, const void* x, const void* W_router,
-                 const float* expert_bias, const void* W_gate, const void* W_up, const void* W_down,
-                 const void* W_shared_gate, const void* W_shared_up, const void* W_shared_down, int score_fn,
-                 int norm_topk, float route_scale, void* out, int32_t* topk_idx, float* topk_w, char* ws,
-                 cudaStream_t st) {
-  int rc = run_route(p, di, x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w, ws, st);
-  if (rc == MOE_OK) rc = launch_permute(p, topk_idx, topk_w, ws, st);
+// Steps a3..a7 on a routing already in topk_idx / topk_w.
+int experts_impl(const Plan& p, const DeviceInfo& di, const void* x, const int32_t* topk_idx, const float* topk_w,
+                 const void* W_gate, const void* W_up, const void* W_down, const void* W_shared_gate,
+                 const void* W_shared_up, const void* W_shared_down, const void* W_shared_gate_vec, void* out,
+                 char* ws, cudaStream_t st) {
+  int rc = launch_permute(p, topk_idx, topk_w, ws, st);
   if (rc == MOE_OK) rc = run_gate_up(p, di, x, W_gate, W_up, W_shared_gate, W_shared_up, ws, st);
   if (rc == MOE_OK) rc = run_down(p, di, W_down, W_shared_down, ws, st);
-  if (rc == MOE_OK) rc = launch_combine(p, out, ws, st);
+  if (rc == MOE_OK) rc = launch_combine(p, out, ws, x, W_shared_gate_vec, st);
   return rc;
+}
+
+int forward_impl(const Plan& p, const DeviceInfo& di, const void* x, const void* W_router,
+                 const float* expert_bias, const void* W_gate, const void* W_up, const void* W_down,
+                 const void* W_shared_gate, const void* W_shared_up, const void* W_shared_down,
+                 const void* W_shared_gate_vec, int score_fn, int norm_topk, float route_scale, void* out,
+                 int32_t* topk_idx, float* topk_w, char* ws, cudaStream_t st) {
+  int rc = run_route(p, di, x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w, ws, st);
+  if (rc == MOE_OK)
+    rc = experts_impl(p, di, x, topk_idx, topk_w, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down,
+                      W_shared_gate_vec, out, ws, st);
+  return rc;
+}
+
+int check_gate_vec(const Plan& p, const void* W_shared_gate_vec) {
+  if (!W_shared_gate_vec) return MOE_OK;
+  if (p.S == 0) return MOE_ERR_INVALID_ARG;
+  return aligned16(W_shared_gate_vec) ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -312,6 +329,7 @@ int make_plan(const moe_shape* s, Plan* p) {
   q.ostage = take(static_cast<size_t>(T) * d * 2);
   q.istage = take(static_cast<size_t>(T) * k * 4);
   q.wstage = take(static_cast<size_t>(T) * k * 4);
+  q.sgate = take(static_cast<size_t>(T) * (S > 0 ? S : 1) * 4);
   q.total = off;
   *p = q;
   return MOE_OK;
@@ -425,23 +443,49 @@ int moe_expert_down(const moe_shape* shape, const void* W_down, const void* W_sh
   return run_down(p, di, W_down, W_shared_down, static_cast<char*>(workspace), as_stream(stream));
 }
 
-int moe_combine(const moe_shape* shape, void* out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+int moe_combine(const moe_shape* shape, const void* x, const void* W_shared_gate_vec, void* out, void* workspace,
+                size_t workspace_bytes, moe_stream_t stream) {
   Plan p;
   int rc = make_plan(shape, &p);
   if (rc != MOE_OK) return rc;
   if (!out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(out)) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_gate_vec(p, W_shared_gate_vec)) != MOE_OK) return rc;
+  if (W_shared_gate_vec && !x) return MOE_ERR_INVALID_ARG;
+  if (W_shared_gate_vec && !aligned16(x)) return MOE_ERR_UNSUPPORTED;
   if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
   DeviceInfo di;
   if ((rc = check_device(&di)) != MOE_OK) return rc;
-  return launch_combine(p, out, static_cast<const char*>(workspace), as_stream(stream));
+  return launch_combine(p, out, static_cast<char*>(workspace), x, W_shared_gate_vec, as_stream(stream));
+}
+
+int moe_experts_forward(const moe_shape* shape, const void* x, const int32_t* topk_idx, const float* topk_w,
+                        const void* W_gate, const void* W_up, const void* W_down, const void* W_shared_gate,
+                        const void* W_shared_up, const void* W_shared_down, const void* W_shared_gate_vec, void* out,
+                        void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if (!x || !topk_idx || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(topk_idx) || !aligned16(topk_w) || !aligned16(out)) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_expert_args(p, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down)) != MOE_OK)
+    return rc;
+  if ((rc = check_gate_vec(p, W_shared_gate_vec)) != MOE_OK) return rc;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = as_stream(stream);
+  if (cudaMemsetAsync(ws + p.err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+  return experts_impl(p, di, x, topk_idx, topk_w, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down,
+                      W_shared_gate_vec, out, ws, st);
 }
 
 int moe_forward(const moe_shape* shape, const void* x, const void* W_router, const float* expert_bias,
                 const void* W_gate, const void* W_up, const void* W_down, const void* W_shared_gate,
-                const void* W_shared_up, const void* W_shared_down, int score_fn, int norm_topk, float route_scale,
-                void* out, int32_t* topk_idx, float* topk_w, void* workspace, size_t workspace_bytes,
-                moe_stream_t stream) {
+                const void* W_shared_up, const void* W_shared_down, const void* W_shared_gate_vec, int score_fn,
+                int norm_topk, float route_scale, void* out, int32_t* topk_idx, float* topk_w, void* workspace,
+                size_t workspace_bytes, moe_stream_t stream) {
   Plan p;
   int rc = make_plan(shape, &p);
   if (rc != MOE_OK) return rc;
@@ -451,19 +495,20 @@ int moe_forward(const moe_shape* shape, const void* x, const void* W_router, con
     return rc;
   if (!out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(out)) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_gate_vec(p, W_shared_gate_vec)) != MOE_OK) return rc;
   if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
   DeviceInfo di;
   if ((rc = check_device(&di)) != MOE_OK) return rc;
   return forward_impl(p, di, x, W_router, expert_bias, W_gate, W_up, W_down, W_shared_gate, W_shared_up,
-                      W_shared_down, score_fn, norm_topk, route_scale, out, topk_idx, topk_w,
+                      W_shared_down, W_shared_gate_vec, score_fn, norm_topk, route_scale, out, topk_idx, topk_w,
                       static_cast<char*>(workspace), as_stream(stream));
 }
 
 int moe_forward_host(const moe_shape* shape, const void* x_host, const void* W_router, const float* expert_bias,
                      const void* W_gate, const void* W_up, const void* W_down, const void* W_shared_gate,
-                     const void* W_shared_up, const void* W_shared_down, int score_fn, int norm_topk,
-                     float route_scale, void* out_host, int32_t* topk_idx_host, float* topk_w_host,
-                     void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+                     const void* W_shared_up, const void* W_shared_down, const void* W_shared_gate_vec,
+                     int score_fn, int norm_topk, float route_scale, void* out_host, int32_t* topk_idx_host,
+                     float* topk_w_host, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
   Plan p;
   int rc = make_plan(shape, &p);
   if (rc != MOE_OK) return rc;
@@ -478,6 +523,7 @@ int moe_forward_host(const moe_shape* shape, const void* x_host, const void* W_r
     return rc;
   if ((rc = check_expert_args(p, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down)) != MOE_OK)
     return rc;
+  if ((rc = check_gate_vec(p, W_shared_gate_vec)) != MOE_OK) return rc;
   DeviceInfo di;
   if ((rc = check_device(&di)) != MOE_OK) return rc;
   cudaStream_t st = as_stream(stream);
@@ -485,7 +531,7 @@ int moe_forward_host(const moe_shape* shape, const void* x_host, const void* W_r
   const size_t tkbytes = static_cast<size_t>(p.T) * p.k * 4;
   if (cudaMemcpyAsync(xd, x_host, xbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
   rc = forward_impl(p, di, xd, W_router, expert_bias, W_gate, W_up, W_down, W_shared_gate, W_shared_up,
-                    W_shared_down, score_fn, norm_topk, route_scale, od, id, wd, ws, st);
+                    W_shared_down, W_shared_gate_vec, score_fn, norm_topk, route_scale, od, id, wd, ws, st);
   if (rc != MOE_OK) return rc;
   if (cudaMemcpyAsync(out_host, od, xbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaMemcpyAsync(topk_idx_host, id, tkbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||

@@ -45,7 +45,7 @@ struct Plan {
   int shared_units1, shared_units2;
   // region offsets (bytes)
   size_t err, nunits, logits, blkcnt, counts, roff, perm, roww, inv, units1, units2;
-  size_t Hr, Hs, Yr, Ys, xstage, ostage, istage, wstage;
+  size_t Hr, Hs, Yr, Ys, xstage, ostage, istage, wstage, sgate;
   size_t total;
 };
 
@@ -94,7 +94,8 @@ int launch_topk(const float* logits, const float* bias, int T, int E, int k, int
 int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, char* ws,
                    cudaStream_t st);
 
-int launch_combine(const Plan& p, void* out, const char* ws, cudaStream_t st);
+int launch_combine(const Plan& p, void* out, char* ws, const void* x, const void* shared_gate_vec,
+                   cudaStream_t st);
 
 int launch_wait_timeout(uint32_t* err, uint64_t timeout_ns, cudaStream_t st);
 

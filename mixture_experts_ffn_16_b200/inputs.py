@@ -7,8 +7,9 @@ Recipe (same for every workload):
   * one ``torch.Generator`` on the target device, seeded with the workload's
     seed;
   * draw order: x, W_router, expert_bias, W_gate, W_up, W_down,
-    W_shared_gate, W_shared_up, W_shared_down, then (skewed workload only) the
-    shuffled expert ranks;
+    W_shared_gate, W_shared_up, W_shared_down, then (gated shared expert only)
+    W_shared_gate_vec [S,d], then (skewed workload only) the shuffled expert
+    ranks;
   * each tensor is drawn as fp32 N(0, std) in slabs of at most 2**27 elements
     along its first axis, then rounded to bf16 (expert_bias stays fp32);
   * x ~ N(0, 1); all weights ~ N(0, 0.02); expert_bias ~ N(0, 0.1) where the
@@ -43,6 +44,7 @@ class MoEConfig:
     route_scale: float = 1.0
     bias_std: float = 0.0              # 0 = no expert_bias tensor
     skew: str = ""                     # "" | "zipf_rank"
+    shared_gate: bool = False          # per-token sigmoid gate on the shared experts (Qwen3.5)
     seed: int = 0
     x_std: float = 1.0
     w_std: float = 0.02
@@ -108,6 +110,9 @@ def make_inputs(cfg: MoEConfig, device="cpu", seed=None):
         W_shared_down = _randn_bf16((S, d, fs), cfg.w_std, gen, device)
     else:
         W_shared_gate = W_shared_up = W_shared_down = None
+    W_shared_gate_vec = None
+    if cfg.shared_gate and S > 0:
+        W_shared_gate_vec = _randn_bf16((S, d), cfg.w_std, gen, device)
     ranks = None
     if cfg.skew == "zipf_rank":
         ranks = torch.randperm(E, generator=gen, device=device) + 1
@@ -116,7 +121,7 @@ def make_inputs(cfg: MoEConfig, device="cpu", seed=None):
         W_router[:, 0] = offset.to(torch.bfloat16)
     return dict(x=x, W_router=W_router, expert_bias=bias, W_gate=W_gate, W_up=W_up, W_down=W_down,
                 W_shared_gate=W_shared_gate, W_shared_up=W_shared_up, W_shared_down=W_shared_down,
-                ranks=ranks)
+                W_shared_gate_vec=W_shared_gate_vec, ranks=ranks)
 
 
 def bf16_bits(t):
@@ -139,7 +144,8 @@ def oracle_args(inp):
                 W_shared_gate=bf16_bits(inp["W_shared_gate"]),
                 W_shared_up=bf16_bits(inp["W_shared_up"]),
                 W_shared_down=bf16_bits(inp["W_shared_down"]),
-                expert_bias=host_f32(inp["expert_bias"]))
+                expert_bias=host_f32(inp["expert_bias"]),
+                shared_gate=bf16_bits(inp.get("W_shared_gate_vec")))
 
 
 def from_bits(a, device="cpu"):

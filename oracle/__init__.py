@@ -54,7 +54,7 @@ def _load():
             i = ctypes.c_int
             lib.oracle_moe_forward.restype = i
             lib.oracle_moe_forward.argtypes = (
-                [i] * 7 + [P] * 3 + [P] * 6 + [i, i, ctypes.c_double] + [P, i, P, i] + [P] * 8 + [i])
+                [i] * 7 + [P] * 3 + [P] * 6 + [i, i, ctypes.c_double] + [P, i, P, P, P, i] + [P] * 8 + [i])
             _lib = lib
     return _lib
 
@@ -77,8 +77,8 @@ def _u16(a, shape, name):
 def forward(x, W_router, W_gate=None, W_up=None, W_down=None,
             W_shared_gate=None, W_shared_up=None, W_shared_down=None,
             expert_bias=None, *, k, score_fn="softmax", norm_topk=True, route_scale=1.0,
-            tokens=None, forced_idx=None, route_only=False, want_logits=False,
-            n_threads=None):
+            tokens=None, forced_idx=None, forced_w=None, shared_gate=None, route_only=False,
+            want_logits=False, n_threads=None):
     """Run the oracle.
 
     Shapes (bf16 bit patterns as uint16): x [T,d], W_router [E,d],
@@ -88,7 +88,9 @@ def forward(x, W_router, W_gate=None, W_up=None, W_down=None,
     ``tokens`` restricts evaluation to those token ids (outputs are in that
     order); ``forced_idx`` [n,k] replaces the router's choice of experts (the
     weights are then the scores of the forced experts, renormalised the same
-    way).  Returns a dict of float64/int32 numpy arrays: ``out`` [n,d],
+    way) unless ``forced_w`` [n,k] gives the weights as well (external
+    routing).  ``shared_gate`` [S,d] (bf16 bits) scales shared expert s by
+    sigma(shared_gate[s] . x) per token.  Returns a dict of float64/int32 numpy arrays: ``out`` [n,d],
     ``topk_idx`` [n,k], ``topk_w`` [n,k], ``sel_keys`` / ``sel_order`` [n,k+1]
     (selection keys and experts of the first k+1 in selection order; -inf / -1
     past E), and with ``want_logits`` also ``logits``, ``scores`` and the
@@ -125,6 +127,14 @@ def forward(x, W_router, W_gate=None, W_up=None, W_down=None,
     forced = None if forced_idx is None else np.ascontiguousarray(forced_idx, dtype=np.int32)
     if forced is not None and forced.shape != (n, k):
         raise ValueError("forced_idx must be [n_tokens, k]")
+    fw = None if forced_w is None else np.ascontiguousarray(forced_w, dtype=np.float64)
+    if fw is not None and (forced is None or fw.shape != (n, k)):
+        raise ValueError("forced_w needs forced_idx and must be [n_tokens, k]")
+    sg = None
+    if shared_gate is not None:
+        if route_only or S == 0:
+            raise ValueError("shared_gate needs shared experts")
+        sg = _u16(shared_gate, (S, d), "shared_gate")
 
     out = None if route_only else np.zeros((n, d), np.float64)
     topk_idx = np.zeros((n, k), np.int32)
@@ -143,7 +153,7 @@ def forward(x, W_router, W_gate=None, W_up=None, W_down=None,
         _ptr(W_shared_gate), _ptr(W_shared_up), _ptr(W_shared_down),
         SCORE_FNS[score_fn] if isinstance(score_fn, str) else int(score_fn),
         int(bool(norm_topk)), float(route_scale),
-        _ptr(tok), n, _ptr(forced), int(bool(route_only)),
+        _ptr(tok), n, _ptr(forced), _ptr(fw), _ptr(sg), int(bool(route_only)),
         _ptr(out), _ptr(topk_idx), _ptr(topk_w), _ptr(sel_keys), _ptr(sel_order),
         _ptr(logits), _ptr(scores), _ptr(keys), int(n_threads))
     if st != 0:

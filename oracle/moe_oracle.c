@@ -30,7 +30,9 @@
  *   - ties in the top-k order go to the lower expert index;
  *   - the softmax selection key is the softmax probability itself;
  *   - the renormalisation denominator is guarded by max(sum, DBL_MIN);
- *   - the shared experts are ungated (weight 1);
+ *   - the shared experts are ungated (weight 1) unless gate vectors are
+ *     given, then scaled by sigma(w_s . x) per token (qwen3-5-vs-gemma-4,
+ *     component table, Qwen3.5 shared-expert cell);
  *   - experts carry no biases; the block output is residual-free;
  *   - weights follow the [out, in] (nn.Linear) layout:
  *       W_router [E,d], W_gate/W_up [E,f,d], W_down [E,d,f],
@@ -146,6 +148,8 @@ typedef struct {
     const int32_t *tokens;   /* n_tokens token ids, or NULL for 0..n_tokens-1 */
     int n_tokens;
     const int32_t *forced;   /* [n_tokens,k] expert ids to use instead of the router's pick, or NULL */
+    const double *forced_w;  /* [n_tokens,k] combine weights to use as given (with forced), or NULL */
+    const uint16_t *sgate;   /* [S,d] shared-expert gate vectors (bf16), or NULL = ungated */
     int route_only;          /* 1: skip the experts */
     double *out;             /* [n_tokens,d] or NULL */
     int32_t *topk_idx;       /* [n_tokens,k] or NULL */
@@ -167,7 +171,9 @@ typedef struct {
  *     c_e = s_e otherwise (the bias only picks experts)
  *  4. sel = the k largest keys, descending, ties to the lower index
  *  5. w_j = s_{sel_j}; if norm_topk, w_j /= sum_j s_{sel_j}; w_j *= route_scale
- *  6. out = sum_j w_j SwiGLU_{sel_j}(x) + sum_s SwiGLU_shared_s(x) */
+ *     (external routing: the given experts and weights replace 4 and 5)
+ *  6. out = sum_j w_j SwiGLU_{sel_j}(x) + sum_s g_s SwiGLU_shared_s(x),
+ *     g_s = 1, or sigma(w_s . x) with gate vectors */
 static int oracle_token(oracle_job *J, int n, double *logit, double *s, keyed *kv,
                         double *h, double *y)
 {
@@ -210,12 +216,17 @@ static int oracle_token(oracle_job *J, int n, double *logit, double *s, keyed *k
     }
 
     double w[64], denom = 0.0;
-    for (int j = 0; j < k; ++j) { w[j] = s[sel[j]]; denom += w[j]; }
-    if (J->norm_topk) {
-        if (denom < DBL_MIN) denom = DBL_MIN;
-        for (int j = 0; j < k; ++j) w[j] /= denom;
+    if (J->forced && J->forced_w) {
+        /* external routing: the caller's weights, as given */
+        for (int j = 0; j < k; ++j) w[j] = J->forced_w[(size_t)n * k + j];
+    } else {
+        for (int j = 0; j < k; ++j) { w[j] = s[sel[j]]; denom += w[j]; }
+        if (J->norm_topk) {
+            if (denom < DBL_MIN) denom = DBL_MIN;
+            for (int j = 0; j < k; ++j) w[j] /= denom;
+        }
+        for (int j = 0; j < k; ++j) w[j] *= J->route_scale;
     }
-    for (int j = 0; j < k; ++j) w[j] *= J->route_scale;
 
     if (J->topk_idx) for (int j = 0; j < k; ++j) J->topk_idx[(size_t)n * k + j] = sel[j];
     if (J->topk_w) for (int j = 0; j < k; ++j) J->topk_w[(size_t)n * k + j] = w[j];
@@ -229,9 +240,19 @@ static int oracle_token(oracle_job *J, int n, double *logit, double *s, keyed *k
                                  w[j], h, y);
     }
     const size_t ssz = (size_t)J->fs * d;
-    for (int sh = 0; sh < J->S; ++sh)
+    for (int sh = 0; sh < J->S; ++sh) {
+        /* shared expert weight: 1 (ungated), or sigma(w_s . x) with the
+         * per-token gate of the Qwen3.5 shared expert */
+        double gw = 1.0;
+        if (J->sgate) {
+            double z = 0.0;
+            const uint16_t *gv = J->sgate + (size_t)sh * d;
+            for (int i = 0; i < d; ++i) z += bf16_to_double(gv[i]) * bf16_to_double(x_t[i]);
+            gw = 1.0 / (1.0 + exp(-z));
+        }
         swiglu_expert_accumulate(d, J->fs, x_t, J->Wsg + sh * ssz, J->Wsu + sh * ssz,
-                                 J->Wsd + sh * ssz, 1.0, h, y);
+                                 J->Wsd + sh * ssz, gw, h, y);
+    }
     memcpy(J->out + (size_t)n * d, y, sizeof(double) * d);
     return 0;
 }
@@ -272,7 +293,7 @@ int oracle_moe_forward(int T, int d, int E, int k, int f, int S, int fs,
                        const uint16_t *Wsg, const uint16_t *Wsu, const uint16_t *Wsd,
                        int score_fn, int norm_topk, double route_scale,
                        const int32_t *tokens, int n_tokens, const int32_t *forced,
-                       int route_only,
+                       const double *forced_w, const uint16_t *sgate, int route_only,
                        double *out, int32_t *topk_idx, double *topk_w, double *sel_keys,
                        int32_t *sel_order, double *logits_out, double *scores_out, double *keys_out,
                        int n_threads)
@@ -291,6 +312,7 @@ int oracle_moe_forward(int T, int d, int E, int k, int f, int S, int fs,
     J.Wg = Wg; J.Wu = Wu; J.Wd = Wd; J.Wsg = Wsg; J.Wsu = Wsu; J.Wsd = Wsd;
     J.score_fn = score_fn; J.norm_topk = norm_topk; J.route_scale = route_scale;
     J.tokens = tokens; J.n_tokens = n_tokens; J.forced = forced; J.route_only = route_only;
+    J.forced_w = forced_w; J.sgate = sgate;
     J.out = out; J.topk_idx = topk_idx; J.topk_w = topk_w; J.sel_keys = sel_keys;
     J.sel_order = sel_order;
     J.logits_out = logits_out; J.scores_out = scores_out; J.keys_out = keys_out;

@@ -76,7 +76,7 @@ def test_invalid_shapes(lib, bad, code):
     base.update(bad)
     s = api.make_shape(**base)
     assert api.moe_workspace_bytes(s) == 0
-    st = lib.moe_forward(ctypes.byref(s), *([ctypes.c_void_p(256)] * 9), 0, 1, 1.0,
+    st = lib.moe_forward(ctypes.byref(s), *([ctypes.c_void_p(256)] * 9), None, 0, 1, 1.0,
                          *([ctypes.c_void_p(256)] * 4), 1 << 30, None)
     assert st == code
 
@@ -87,26 +87,33 @@ def test_argument_checks_before_any_device_work(lib):
     P = ctypes.c_void_p
     good = [P(4096)] * 9
     # null x
-    st = lib.moe_forward(ctypes.byref(s), None, *good[1:], 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096),
+    st = lib.moe_forward(ctypes.byref(s), None, *good[1:], None, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096),
                          n, None)
     assert st == api.MOE_ERR_INVALID_ARG
     # bad score function / norm flag / non-finite scale
     for sf, nt, sc in [(3, 1, 1.0), (0, 2, 1.0), (0, 1, float("inf"))]:
-        st = lib.moe_forward(ctypes.byref(s), *good, sf, nt, sc, P(4096), P(4096), P(4096), P(4096), n, None)
+        st = lib.moe_forward(ctypes.byref(s), *good, None, sf, nt, sc, P(4096), P(4096), P(4096), P(4096), n, None)
         assert st == api.MOE_ERR_INVALID_ARG
     # misaligned pointer
-    st = lib.moe_forward(ctypes.byref(s), P(4098), *good[1:], 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096),
+    st = lib.moe_forward(ctypes.byref(s), P(4098), *good[1:], None, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096),
                          n, None)
     assert st == api.MOE_ERR_UNSUPPORTED
     # shared weights given with S == 0
     s0 = api.make_shape(16, 128, 8, 2, 128, 0, 0)
-    st = lib.moe_forward(ctypes.byref(s0), *good, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096),
+    st = lib.moe_forward(ctypes.byref(s0), *good, None, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096),
                          api.moe_workspace_bytes(s0), None)
     assert st == api.MOE_ERR_INVALID_ARG
+    # shared-expert gate vector given with S == 0, or misaligned
+    st = lib.moe_forward(ctypes.byref(s0), *good[:6], None, None, None, P(4096), 0, 1, 1.0,
+                         P(4096), P(4096), P(4096), P(4096), api.moe_workspace_bytes(s0), None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    st = lib.moe_forward(ctypes.byref(s), *good, P(4100), 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096),
+                         n, None)
+    assert st == api.MOE_ERR_UNSUPPORTED
     # workspace too small / misaligned
-    st = lib.moe_forward(ctypes.byref(s), *good, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096), n - 1, None)
+    st = lib.moe_forward(ctypes.byref(s), *good, None, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4096), n - 1, None)
     assert st == api.MOE_ERR_WORKSPACE
-    st = lib.moe_forward(ctypes.byref(s), *good, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4128), n, None)
+    st = lib.moe_forward(ctypes.byref(s), *good, None, 0, 1, 1.0, P(4096), P(4096), P(4096), P(4128), n, None)
     assert st == api.MOE_ERR_WORKSPACE
 
 
@@ -121,3 +128,26 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(api, "_lib", None)
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         api.load()
+
+
+def test_experts_forward_argument_checks(lib):
+    """External-indices entry: null or misaligned routing arrays and a gate
+    vector with no shared expert are refused before any device work."""
+    s = api.make_shape(16, 128, 8, 2, 128, 1, 128)
+    n = api.moe_workspace_bytes(s)
+    P = ctypes.c_void_p
+    w6 = [P(4096)] * 6
+
+    def call(shape=s, x=P(4096), idx=P(4096), wt=P(4096), gv=None, out=P(4096), ws_bytes=n, weights=w6):
+        return lib.moe_experts_forward(ctypes.byref(shape), x, idx, wt, *weights, gv, out, P(4096), ws_bytes, None)
+
+    assert call(idx=None) == api.MOE_ERR_INVALID_ARG
+    assert call(wt=None) == api.MOE_ERR_INVALID_ARG
+    assert call(out=None) == api.MOE_ERR_INVALID_ARG
+    assert call(idx=P(4100)) == api.MOE_ERR_UNSUPPORTED
+    assert call(gv=P(4104)) == api.MOE_ERR_UNSUPPORTED
+    assert call(weights=w6[:3] + [None] * 3) == api.MOE_ERR_INVALID_ARG
+    s0 = api.make_shape(16, 128, 8, 2, 128, 0, 0)
+    assert call(shape=s0, weights=w6[:3] + [None] * 3, gv=P(4096),
+                ws_bytes=api.moe_workspace_bytes(s0)) == api.MOE_ERR_INVALID_ARG
+    assert call(ws_bytes=n - 1) == api.MOE_ERR_WORKSPACE

@@ -161,7 +161,7 @@ def test_error_codes_enqueue_nothing(case):
                                ctypes.c_void_p(inp["W_down"].data_ptr()),
                                ctypes.c_void_p(inp["W_shared_gate"].data_ptr()),
                                ctypes.c_void_p(inp["W_shared_up"].data_ptr()),
-                               ctypes.c_void_p(inp["W_shared_down"].data_ptr()), score, 1, 1.0,
+                               ctypes.c_void_p(inp["W_shared_down"].data_ptr()), None, score, 1, 1.0,
                                ctypes.c_void_p(out_t.data_ptr()), ctypes.c_void_p(layer.topk_idx.data_ptr()),
                                ctypes.c_void_p(layer.topk_w.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
                                ws.numel() if ws_bytes is None else ws_bytes, None)

@@ -124,3 +124,53 @@ def test_full_size_workloads_sampled(oracle_mod, name, n_tok):
     host = oracle_args(inp)
     rep = check_parity(oracle_mod, cfg, host, out[tokens], idx[tokens], w[tokens], tokens=tokens)
     print(name, rep)
+
+
+GATED = [
+    MoEConfig("qwen_like_gated_shared", T=300, d=512, E=64, k=10, f=128, S=1, fs=256, shared_gate=True, seed=24),
+    MoEConfig("gated_two_shared_sigmoid", T=150, d=256, E=16, k=4, f=64, S=2, fs=128, shared_gate=True,
+              score_fn="sigmoid", bias_std=0.1, seed=25),
+]
+
+
+@pytest.mark.parametrize("cfg", GATED, ids=lambda c: c.name)
+def test_gated_shared_expert_every_token(oracle_mod, cfg):
+    """The Qwen3.5 shared expert: scaled per token by sigmoid(w . x) before it
+    is added to the routed sum."""
+    rep, _ = parity_case(oracle_mod, cfg)
+    assert rep["tokens"] == cfg.T
+
+
+def test_gated_shared_full_size_sampled(oracle_mod):
+    cfg = MoEConfig("prefill_softmax_gated", T=4096, d=2048, E=256, k=8, f=512, S=1, fs=512, shared_gate=True,
+                    seed=26)
+    rep, _ = parity_case(oracle_mod, cfg, tokens=_sample(cfg.T, 256, seed=7))
+    assert rep["tokens"] == 256
+
+
+@pytest.mark.parametrize("cfg", [MEDIUM[0], MEDIUM[1], MoEConfig(
+    "external_gated", T=333, d=256, E=24, k=5, f=128, S=1, fs=64, shared_gate=True, seed=27)],
+    ids=lambda c: c.name)
+def test_external_routing_matches_oracle(oracle_mod, cfg):
+    """External-indices mode: the caller's experts and weights (seeded, not the
+    router's) through moe_experts_forward, against the oracle given the same
+    routing."""
+    _need_gpu()
+    inp = make_inputs(cfg, device="cuda")
+    g = torch.Generator().manual_seed(cfg.seed + 500)
+    idx = torch.stack([torch.randperm(cfg.E, generator=g)[:cfg.k] for _ in range(cfg.T)]).to(torch.int32)
+    w = torch.rand((cfg.T, cfg.k), generator=g, dtype=torch.float32) * 2.0 - 0.5
+    shape = api.shape_of(cfg)
+    ws = api.alloc_workspace(shape)
+    out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    api.moe_experts_forward(shape, inp["x"], idx.cuda(), w.cuda(), inp["W_gate"], inp["W_up"], inp["W_down"],
+                            inp["W_shared_gate"], inp["W_shared_up"], inp["W_shared_down"], out, ws,
+                            W_shared_gate_vec=inp.get("W_shared_gate_vec"))
+    assert api.moe_device_status(ws) == api.MOE_OK
+    ref = oracle_mod.forward(**oracle_args(inp), k=cfg.k, forced_idx=idx.numpy(),
+                             forced_w=w.numpy().astype(np.float64))
+    got = out.float().cpu().numpy()
+    scale = np.abs(ref["out"]).max()
+    err = np.abs(got - ref["out"]).max()
+    print(cfg.name, "external routing err ratio", err / scale)
+    assert np.isfinite(got).all() and err <= 2e-2 * scale

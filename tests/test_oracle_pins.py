@@ -374,3 +374,52 @@ def test_keys_are_scores_plus_bias_for_biased_routers(oracle_mod):
         assert np.array_equal(r["keys"], ref)
         np.testing.assert_array_equal(np.take_along_axis(r["keys"], r["sel_order"][:, :3], 1),
                                       r["sel_keys"][:, :3])
+
+
+# ---------------------------------------------------------------- external routing, gated shared expert
+
+def test_external_routing_uses_given_experts_and_weights(oracle_mod):
+    """Given experts and weights replace the router's: the output is the
+    weighted sum of the dense experts with exactly those weights."""
+    rng = np.random.default_rng(20)
+    E, k, S = 7, 3, 1
+    c = rand_case(rng, 9, 32, E, 24, S=S, fs=16)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(9)]).astype(np.int32)
+    w = rng.normal(0, 1, (9, k))
+    r = oracle_mod.forward(**c, k=k, forced_idx=idx, forced_w=w)
+    X = widen(c["x"])
+    ref = swiglu_dense(X, widen(c["W_shared_gate"][0]), widen(c["W_shared_up"][0]),
+                       widen(c["W_shared_down"][0]))
+    for t in range(9):
+        for j in range(k):
+            e = idx[t, j]
+            ref[t] += w[t, j] * swiglu_dense(X[t:t + 1], widen(c["W_gate"][e]), widen(c["W_up"][e]),
+                                             widen(c["W_down"][e]))[0]
+    np.testing.assert_allclose(r["out"], ref, rtol=1e-11, atol=1e-12)
+    assert np.array_equal(r["topk_idx"], idx) and np.array_equal(r["topk_w"], w)
+    # the oracle's own routing given back reproduces its output bit for bit
+    own = oracle_mod.forward(**c, k=k)
+    back = oracle_mod.forward(**c, k=k, forced_idx=own["topk_idx"], forced_w=own["topk_w"])
+    assert np.array_equal(back["out"], own["out"])
+
+
+def test_shared_gate_scales_shared_expert_by_sigmoid(oracle_mod):
+    """Qwen3.5 shared expert: output scaled by sigma(w . x) before it is added.
+    A zero gate vector gives exactly 1/2; otherwise the difference to the
+    ungated block is (sigma(w.x) - 1) * shared expert (numpy / scipy forms)."""
+    rng = np.random.default_rng(21)
+    S, d = 2, 32
+    c = rand_case(rng, 10, d, 5, 16, S=S, fs=24)
+    ungated = oracle_mod.forward(**c, k=2)
+    X = widen(c["x"])
+    shared = [swiglu_dense(X, widen(c["W_shared_gate"][s]), widen(c["W_shared_up"][s]),
+                           widen(c["W_shared_down"][s])) for s in range(S)]
+    zero = oracle_mod.forward(**c, k=2, shared_gate=bits(np.zeros((S, d))))
+    np.testing.assert_allclose(zero["out"], ungated["out"] - 0.5 * (shared[0] + shared[1]),
+                               rtol=1e-11, atol=1e-12)
+    gv = bits(rng.normal(0, 0.3, (S, d)))
+    g = oracle_mod.forward(**c, k=2, shared_gate=gv)
+    gates = expit(X @ widen(gv).T)          # [T, S]
+    ref = ungated["out"] + sum((gates[:, s:s + 1] - 1.0) * shared[s] for s in range(S))
+    np.testing.assert_allclose(g["out"], ref, rtol=1e-11, atol=1e-12)
+    assert np.array_equal(g["topk_idx"], ungated["topk_idx"])
