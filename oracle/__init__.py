@@ -55,6 +55,10 @@ def _load():
             lib.oracle_moe_forward.restype = i
             lib.oracle_moe_forward.argtypes = (
                 [i] * 7 + [P] * 3 + [P] * 6 + [i, i, ctypes.c_double] + [P, i, P, P, P, i] + [P] * 8 + [i])
+            lib.oracle_rmsnorm.restype = i
+            lib.oracle_rmsnorm.argtypes = [i, i, P, P, ctypes.c_double, P, P]
+            lib.oracle_double_to_bf16.restype = ctypes.c_uint16
+            lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
             _lib = lib
     return _lib
 
@@ -175,3 +179,34 @@ def rel_gap(a, b):
     with np.errstate(invalid="ignore", divide="ignore"):
         g = np.where(m > 0, np.abs(a - b) / np.where(m > 0, m, 1.0), 0.0)
     return g
+
+
+def to_bf16_bits(values):
+    """fp64 values -> raw bf16 bits (nearest, ties to even), element by element."""
+    lib = _load()
+    v = np.asarray(values, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    flat, of = v.ravel(), out.ravel()
+    for n in range(flat.size):
+        of[n] = lib.oracle_double_to_bf16(float(flat[n]))
+    return out
+
+
+def rmsnorm(x, gain, eps):
+    """Pre-norm RMSNorm with zero-centred gains: y = x / sqrt(mean(x^2) + eps) * (1 + g).
+
+    x: [T, d] raw bf16 bits (uint16); gain: [d] raw bf16 bits; eps: float.
+    Returns {"y": fp64 [T, d], "y_bits": bf16 bits [T, d] (y rounded to nearest even)}.
+    """
+    lib = _load()
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16 or x.ndim != 2:
+        raise TypeError("x: expected [T, d] raw bf16 bits (uint16)")
+    T, d = x.shape
+    gain = _u16(gain, (d,), "gain")
+    y = np.empty((T, d), dtype=np.float64)
+    yb = np.empty((T, d), dtype=np.uint16)
+    rc = lib.oracle_rmsnorm(T, d, _ptr(x), _ptr(gain), float(eps), _ptr(y), _ptr(yb))
+    if rc != 0:
+        raise ValueError(f"oracle_rmsnorm: invalid arguments ({rc})")
+    return {"y": y, "y_bits": yb}

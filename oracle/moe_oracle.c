@@ -329,3 +329,60 @@ int oracle_moe_forward(int T, int d, int E, int k, int f, int S, int fs,
     pthread_mutex_destroy(&J.mu);
     return J.status;
 }
+
+/* ------------------------------------------------------------------ RMSNorm
+ * The pre-norm RMSNorm that produces the block's input (qwen3-5-vs-deepseek-v4,
+ * Qwen3.5 diagram: "RMSNorm - pre-norm" directly before the router), with
+ * zero-centred gains (same page, component table, Qwen3.5 residual-stream
+ * cell): the stored gain g is centred on zero, so the scale applied is 1 + g.
+ *
+ *   y[t,i] = x[t,i] / sqrt(mean_j x[t,j]^2 + eps) * (1 + g[i])
+ *
+ * in double, then rounded to bf16 (nearest, ties to even) because the block
+ * takes bf16 input.  eps is not given on the pages; the caller passes it. */
+
+/* double -> bf16 bits, round to nearest, ties to even, straight from the
+ * double (no intermediate float rounding).  bf16 keeps 8 significant bits; a
+ * value in [2^(e-1), 2^e) is rounded to a multiple of 2^(e-8), and below the
+ * smallest normal (2^-126) to a multiple of 2^-133.  The rounded value is
+ * exactly representable in binary32, whose top 16 bits are the bf16. */
+uint16_t oracle_double_to_bf16(double v)
+{
+    if (isnan(v)) return 0x7FC0;
+    const uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80);
+    int e;
+    frexp(a, &e);                       /* a = m * 2^e, 0.5 <= m < 1 */
+    int qe = e - 8;
+    if (qe < -133) qe = -133;
+    double q = nearbyint(ldexp(a, -qe)); /* exact scaling; default mode = ties to even */
+    double r = ldexp(q, qe);
+    if (r >= 0x1p128) return (uint16_t)(sign | 0x7F80);
+    float f = (float)r;                 /* exact */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | (u >> 16));
+}
+
+int oracle_rmsnorm(int T, int d, const uint16_t *x, const uint16_t *gain, double eps,
+                   double *y, uint16_t *y_bf16)
+{
+    if (T < 0 || d < 1 || !x || !gain || !(eps >= 0.0)) return -1;
+    for (int t = 0; t < T; ++t) {
+        const uint16_t *xr = x + (size_t)t * d;
+        double ss = 0.0;
+        for (int i = 0; i < d; ++i) {
+            const double v = bf16_to_double(xr[i]);
+            ss += v * v;
+        }
+        const double rstd = 1.0 / sqrt(ss / d + eps);
+        for (int i = 0; i < d; ++i) {
+            const double v = bf16_to_double(xr[i]) * rstd * (1.0 + bf16_to_double(gain[i]));
+            if (y) y[(size_t)t * d + i] = v;
+            if (y_bf16) y_bf16[(size_t)t * d + i] = oracle_double_to_bf16(v);
+        }
+    }
+    return 0;
+}

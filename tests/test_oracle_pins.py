@@ -423,3 +423,78 @@ def test_shared_gate_scales_shared_expert_by_sigmoid(oracle_mod):
     ref = ungated["out"] + sum((gates[:, s:s + 1] - 1.0) * shared[s] for s in range(S))
     np.testing.assert_allclose(g["out"], ref, rtol=1e-11, atol=1e-12)
     assert np.array_equal(g["topk_idx"], ungated["topk_idx"])
+
+
+# ---------------------------------------------------------------- pre-norm RMSNorm
+# y = x / sqrt(mean(x^2) + eps) * (1 + g), zero-centred gains (qwen3-5-vs-deepseek-v4,
+# Qwen3.5 diagram "RMSNorm - pre-norm" and the residual-stream cell), rounded to bf16.
+
+@pytest.mark.parametrize("v,expect", [
+    (1.0, 0x3F80), (-2.0, 0xC000), (0.0, 0x0000), (-0.0, 0x8000),
+    (1 + 2 ** -8, 0x3F80),                 # halfway, even neighbour below
+    (1 + 3 * 2 ** -8, 0x3F82),             # halfway, even neighbour above
+    (1 + 2 ** -8 + 2 ** -40, 0x3F81),      # just above halfway: not a tie
+    (-(1 + 2 ** -8), 0xBF80),
+    (2 ** 128 - 2 ** 119, 0x7F80),         # halfway between the largest bf16 and 2^128: to even = inf
+    (2 ** 128 - 2 ** 119 - 2 ** 100, 0x7F7F),
+    (2.0 ** -133, 0x0001), (1.5 * 2.0 ** -133, 0x0002), (2.0 ** -134, 0x0000),
+    (2.0 ** -126, 0x0080),
+])
+def test_bf16_rounding_hand_cases(oracle_mod, v, expect):
+    assert int(oracle_mod.to_bf16_bits([v])[0]) == expect
+
+
+def test_bf16_rounding_matches_torch_on_binary32_values(oracle_mod):
+    """For values exact in binary32, nearest-even to bf16 is torch's float->bfloat16 cast."""
+    import torch
+    rng = np.random.default_rng(5)
+    v = np.concatenate([rng.normal(0, 1, 3000), rng.normal(0, 1e-30, 500), rng.normal(0, 1e30, 500)])
+    v = v.astype(np.float32)
+    # plant exact ties: low 16 bits = 0x8000
+    u = v[:400].view(np.uint32) & np.uint32(0xFFFF0000) | np.uint32(0x8000)
+    v[:400] = u.view(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle_mod.to_bf16_bits(v.astype(np.float64))
+    assert np.array_equal(got, ref)
+
+
+def test_rmsnorm_worked_example(oracle_mod):
+    """x = (3, 4), g = 0, eps = 0: mean square 12.5, y = (3, 4) / sqrt(12.5)
+    = (0.848528..., 1.131370...), bf16 0x3F59 (0.84765625) and 0x3F91 (1.1328125)."""
+    x = np.array([[0x4040, 0x4080]], np.uint16)      # 3.0, 4.0
+    r = oracle_mod.rmsnorm(x, np.zeros(2, np.uint16), 0.0)
+    np.testing.assert_allclose(r["y"][0], [3 / math.sqrt(12.5), 4 / math.sqrt(12.5)], rtol=1e-15)
+    assert [int(b) for b in r["y_bits"][0]] == [0x3F59, 0x3F91]
+
+
+def test_rmsnorm_unit_rms_and_power_of_two_invariance(oracle_mod):
+    rng = np.random.default_rng(6)
+    x = bits(rng.normal(0, 3, (7, 96)))
+    g0 = np.zeros(96, np.uint16)
+    r = oracle_mod.rmsnorm(x, g0, 0.0)
+    np.testing.assert_allclose((r["y"] ** 2).mean(1), 1.0, rtol=1e-13)
+    # x * 8 is exact in bf16 (exponent + 3): with eps = 0 every result bit is unchanged
+    x8 = bits(widen(x) * 8)
+    r8 = oracle_mod.rmsnorm(x8, g0, 0.0)
+    assert np.array_equal(r8["y"], r["y"]) and np.array_equal(r8["y_bits"], r["y_bits"])
+
+
+def test_rmsnorm_gain_is_zero_centred(oracle_mod):
+    rng = np.random.default_rng(7)
+    x = bits(rng.normal(0, 1, (5, 64)))
+    base = oracle_mod.rmsnorm(x, np.zeros(64, np.uint16), 1e-6)["y"]
+    minus_one = oracle_mod.rmsnorm(x, np.full(64, 0xBF80, np.uint16), 1e-6)["y"]     # g = -1
+    plus_one = oracle_mod.rmsnorm(x, np.full(64, 0x3F80, np.uint16), 1e-6)["y"]      # g = +1
+    assert not minus_one.any()
+    assert np.array_equal(plus_one, 2 * base)
+    g = bits(rng.normal(0, 0.1, 64))
+    np.testing.assert_allclose(oracle_mod.rmsnorm(x, g, 1e-6)["y"], base * (1 + widen(g)), rtol=1e-15)
+
+
+def test_rmsnorm_eps_closed_form_and_zero_row(oracle_mod):
+    """A constant row c: y = c / sqrt(c^2 + eps); a zero row stays zero."""
+    x = np.array([[0x3E80] * 32, [0] * 32], np.uint16)   # 0.25, 0
+    eps = 0.01
+    r = oracle_mod.rmsnorm(x, np.zeros(32, np.uint16), eps)
+    np.testing.assert_allclose(r["y"][0], 0.25 / math.sqrt(0.0625 + eps), rtol=1e-15)
+    assert not r["y"][1].any() and not r["y_bits"][1].any()
