@@ -59,6 +59,10 @@ def _load():
             lib.oracle_rmsnorm.argtypes = [i, i, P, P, ctypes.c_double, P, P]
             lib.oracle_double_to_bf16.restype = ctypes.c_uint16
             lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
+            lib.oracle_e4m3_to_double.restype = ctypes.c_double
+            lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+            lib.oracle_dequant_mxfp8.restype = i
+            lib.oracle_dequant_mxfp8.argtypes = [i, i, i, P, P, P]
             _lib = lib
     return _lib
 
@@ -210,3 +214,28 @@ def rmsnorm(x, gain, eps):
     if rc != 0:
         raise ValueError(f"oracle_rmsnorm: invalid arguments ({rc})")
     return {"y": y, "y_bits": yb}
+
+
+def e4m3_value(code):
+    """Value of one E4M3 (OCP E4M3FN) code, as a Python float."""
+    return float(_load().oracle_e4m3_to_double(int(code) & 0xFF))
+
+
+def dequant_mxfp8(q, scale):
+    """Block-scaled FP8 weights -> raw bf16 bits.
+
+    q: uint8 [G, rows, K] E4M3 codes; scale: uint8 [G, K/32, rows] UE8M0
+    exponents (2^(s-127)) of the 32-element blocks along K.  Raises if a value
+    is NaN or has no exact bf16 form."""
+    q = np.ascontiguousarray(q)
+    scale = np.ascontiguousarray(scale)
+    if q.dtype != np.uint8 or scale.dtype != np.uint8 or q.ndim != 3:
+        raise TypeError("q: uint8 [G, rows, K]; scale: uint8 [G, K/32, rows]")
+    G, rows, K = q.shape
+    if K % 32 or scale.shape != (G, K // 32, rows):
+        raise ValueError(f"scale: expected shape {(G, K // 32, rows)}, got {scale.shape}")
+    out = np.empty((G, rows, K), dtype=np.uint16)
+    rc = _load().oracle_dequant_mxfp8(G, rows, K, _ptr(q), _ptr(scale), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_dequant_mxfp8: {'bad arguments' if rc == -1 else 'value without an exact bf16 form'}")
+    return out

@@ -386,3 +386,48 @@ int oracle_rmsnorm(int T, int d, const uint16_t *x, const uint16_t *gain, double
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ FP8 weights
+ * Block-scaled FP8 expert weights (the pages name an official FP8 weight
+ * release and "block-scaled FP8": qwen3-5-vs-gemma-4, component table,
+ * Qwen3.5 routed-experts cell; qwen3-5-vs-deepseek-v4, blueprint diagram).
+ * The pages give no block size or scale format.  Reading: OCP MX-style
+ * blocks of 32 consecutive elements along the input dimension K, each with
+ * one power-of-two scale stored as an unbiased-exponent byte (UE8M0):
+ *   w[g, r, c] = e4m3(q[g, r, c]) * 2^(s[g, c / 32, r] - 127)
+ * Scales are stored block-major ([G, K/32, rows]).
+ *
+ * E4M3 (the OCP "E4M3FN" encoding): 1 sign bit, 4 exponent bits with bias 7,
+ * 3 mantissa bits.  Exponent field 0 is subnormal, m/8 * 2^-6; exponent
+ * field 15 with mantissa 7 is NaN; there are no infinities, so the largest
+ * finite magnitude is 1.75 * 2^8 = 448. */
+double oracle_e4m3_to_double(uint8_t b)
+{
+    const int s = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Dequantises G x rows x K weights to bf16 bits.  Returns 0, -1 for bad
+ * arguments (K not a multiple of 32), or -2 when some value is NaN or not
+ * exactly representable in bf16 (the block then has no exact bf16 form). */
+int oracle_dequant_mxfp8(int G, int rows, int K, const uint8_t *q, const uint8_t *scale, uint16_t *w_bf16)
+{
+    if (G < 0 || rows < 0 || K < 32 || K % 32 != 0 || !q || !scale || !w_bf16) return -1;
+    const int nb = K / 32;
+    for (int g = 0; g < G; ++g)
+        for (int r = 0; r < rows; ++r)
+            for (int c = 0; c < K; ++c) {
+                const uint8_t u = scale[((size_t)g * nb + c / 32) * rows + r];
+                if (u == 255) return -2;
+                const double v = oracle_e4m3_to_double(q[((size_t)g * rows + r) * K + c]) * ldexp(1.0, (int)u - 127);
+                if (isnan(v)) return -2;
+                const uint16_t b = oracle_double_to_bf16(v);
+                if (bf16_to_double(b) != v) return -2;
+                w_bf16[((size_t)g * rows + r) * K + c] = b;
+            }
+    return 0;
+}

@@ -498,3 +498,68 @@ def test_rmsnorm_eps_closed_form_and_zero_row(oracle_mod):
     r = oracle_mod.rmsnorm(x, np.zeros(32, np.uint16), eps)
     np.testing.assert_allclose(r["y"][0], 0.25 / math.sqrt(0.0625 + eps), rtol=1e-15)
     assert not r["y"][1].any() and not r["y_bits"][1].any()
+
+
+# ---------------------------------------------------------------- block-scaled FP8 weights
+# w = e4m3(q) * 2^(s - 127), one UE8M0 scale per 32 elements along K (reading of
+# "block-scaled FP8": qwen3-5-vs-deepseek-v4 blueprint diagram; qwen3-5-vs-gemma-4,
+# Qwen3.5 routed-experts cell).
+
+@pytest.mark.parametrize("code,value", [
+    (0x38, 1.0), (0xB8, -1.0), (0x7E, 448.0), (0xFE, -448.0), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9),
+    (0x08, 2.0 ** -6), (0x40, 2.0), (0x3C, 1.5), (0x00, 0.0),
+])
+def test_e4m3_hand_cases(oracle_mod, code, value):
+    assert oracle_mod.e4m3_value(code) == value
+
+
+def test_e4m3_all_codes_match_torch(oracle_mod):
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float32).numpy().astype(np.float64)
+    got = np.array([oracle_mod.e4m3_value(c) for c in codes])
+    nan = np.isnan(ref)
+    assert nan.sum() == 2 and np.array_equal(np.isnan(got), nan)      # 0x7F, 0xFF
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))  # -0.0 at 0x80
+
+
+def test_mxfp8_dequant_block_indexing(oracle_mod):
+    """Each element takes the scale of its own 32-wide block of its own row:
+    distinct scales per (row, block) expose a transposed or shifted index."""
+    G, rows, K = 2, 3, 96
+    q = np.full((G, rows, K), 0x38, np.uint8)                 # every code = 1.0
+    s = np.empty((G, K // 32, rows), np.uint8)
+    for g in range(G):
+        for b in range(K // 32):
+            for r in range(rows):
+                s[g, b, r] = 100 + 10 * g + 3 * b + r
+    w = widen(oracle_mod.dequant_mxfp8(q, s))
+    for g in range(G):
+        for r in range(rows):
+            for c in range(K):
+                assert w[g, r, c] == 2.0 ** (100 + 10 * g + 3 * (c // 32) + r - 127)
+
+
+def test_mxfp8_dequant_random_codes_closed_form(oracle_mod):
+    import torch
+    rng = np.random.default_rng(8)
+    G, rows, K = 3, 5, 64
+    q = rng.integers(0, 256, (G, rows, K)).astype(np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x30                              # no NaN codes
+    s = rng.integers(100, 140, (G, K // 32, rows)).astype(np.uint8)
+    vals = torch.from_numpy(q).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    scale = np.exp2(s.astype(np.float64) - 127)               # [G, K/32, rows]
+    expect = vals * np.repeat(scale.transpose(0, 2, 1), 32, axis=2)
+    assert np.array_equal(widen(oracle_mod.dequant_mxfp8(q, s)), expect)
+
+
+def test_mxfp8_dequant_rejects_nan_and_bad_shapes(oracle_mod):
+    q = np.full((1, 2, 32), 0x38, np.uint8)
+    with pytest.raises(ValueError):
+        oracle_mod.dequant_mxfp8(q, np.full((1, 1, 2), 255, np.uint8))     # NaN scale
+    q[0, 1, 3] = 0x7F
+    with pytest.raises(ValueError):
+        oracle_mod.dequant_mxfp8(q, np.full((1, 1, 2), 127, np.uint8))     # NaN code
+    with pytest.raises(ValueError):
+        oracle_mod.dequant_mxfp8(q, np.full((1, 2, 1), 127, np.uint8))     # row-major scale shape
