@@ -135,6 +135,36 @@ MOE_API int moe_forward_host(const moe_shape *shape,
                      void *out_host, int32_t *topk_idx_host, float *topk_w_host,
                      void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
+/* The block with its pre-norm RMSNorm fused in front (the Qwen3.5 block puts
+ * "RMSNorm - pre-norm" directly before the router: qwen3-5-vs-deepseek-v4,
+ * Qwen3.5 diagram; the gains are zero-centred: same page, component table,
+ * Qwen3.5 residual-stream cell).
+ *   x         [T,d] bf16: the residual stream (not normalised).
+ *   norm_gain [d] bf16: zero-centred gains g; the scale applied is 1 + g.
+ *   norm_eps  finite, >= 0 (the pages give no value; Qwen-family models use
+ *             1e-6).
+ * Runs moe_rmsnorm into the workspace (region MOE_WS_X_STAGE) and then the
+ * block on the normalised rows, which are also what the router, the experts
+ * and the shared-expert gate see.  Everything else as in moe_forward. */
+MOE_API int moe_forward_prenorm(const moe_shape *shape,
+                const void *x, const void *norm_gain, float norm_eps,
+                const void *W_router, const float *expert_bias,
+                const void *W_gate, const void *W_up, const void *W_down,
+                const void *W_shared_gate, const void *W_shared_up, const void *W_shared_down,
+                const void *W_shared_gate_vec,
+                int score_fn, int norm_topk, float route_scale,
+                void *out, int32_t *topk_idx, float *topk_w,
+                void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* Pre-norm RMSNorm alone:
+ *   x_norm[t,i] = bf16( x[t,i] / sqrt(mean_j x[t,j]^2 + eps) * (1 + norm_gain[i]) )
+ * computed in double and rounded to bf16 once (nearest, ties to even).
+ * Only T and d of the shape are used, but the whole shape must be valid.
+ * x, x_norm: bf16 [T,d] device buffers (may not overlap); norm_gain bf16 [d].
+ * Returns MOE_ERR_INVALID_ARG for a null pointer or eps < 0 / not finite. */
+MOE_API int moe_rmsnorm(const moe_shape *shape, const void *x, const void *norm_gain, float eps,
+                void *x_norm, moe_stream_t stream);
+
 /* ---- The steps of moe_forward, callable one by one (same arguments and
  * rules; each step reads what the previous steps left in the workspace, so
  * they must be called in this order with the same shape and workspace). ---- */
@@ -204,6 +234,9 @@ MOE_API int moe_experts_forward(const moe_shape *shape, const void *x, const int
  *   MOE_WS_H_SHARED bf16 [S,Tp,fs]  shared hidden rows, Tp = T rounded up to 16
  *   MOE_WS_Y        bf16 [rows,d]   weighted routed outputs (after moe_expert_down)
  *   MOE_WS_Y_SHARED bf16 [S,Tp,d]   shared outputs
+ *   MOE_WS_X_STAGE  bf16 [T,d]      token rows the library staged: x copied
+ *                                   from the host (moe_forward_host) or the
+ *                                   normalised x (moe_forward_prenorm)
  * Writes the region's byte offset in the workspace and its capacity in bytes.
  * Returns MOE_OK, or MOE_ERR_INVALID_ARG for a bad shape, region or pointer. */
 #define MOE_WS_LOGITS   0
@@ -216,6 +249,7 @@ MOE_API int moe_experts_forward(const moe_shape *shape, const void *x, const int
 #define MOE_WS_H_SHARED 7
 #define MOE_WS_Y        8
 #define MOE_WS_Y_SHARED 9
+#define MOE_WS_X_STAGE  10
 MOE_API int moe_workspace_region(const moe_shape *shape, int region, size_t *offset, size_t *bytes);
 
 /* Synchronises `stream`, then returns MOE_ERR_DEVICE_TIMEOUT if a kernel of a

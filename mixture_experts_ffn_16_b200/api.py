@@ -27,12 +27,12 @@ MOE_ERR_SCRATCH_LIMIT = -6
 SCORE_FNS = {"softmax": 0, "sigmoid": 1, "sqrt_softplus": 2}
 
 WS_REGIONS = {"logits": 0, "counts": 1, "offsets": 2, "perm": 3, "row_w": 4, "inv": 5,
-              "h": 6, "h_shared": 7, "y": 8, "y_shared": 9}
+              "h": 6, "h_shared": 7, "y": 8, "y_shared": 9, "x_stage": 10}
 
 EXPORTED = ["moe_version", "moe_status_string", "moe_workspace_bytes", "moe_forward",
             "moe_forward_host", "moe_route", "moe_permute", "moe_expert_gate_up", "moe_expert_down",
             "moe_combine", "moe_workspace_region", "moe_device_status", "moe_debug_wait_timeout",
-            "moe_route_noalloc", "moe_experts_forward"]
+            "moe_route_noalloc", "moe_experts_forward", "moe_rmsnorm", "moe_forward_prenorm"]
 
 
 class MoEError(RuntimeError):
@@ -72,6 +72,10 @@ def load():
     lib.moe_forward.argtypes = fwd
     lib.moe_forward_host.restype = I
     lib.moe_forward_host.argtypes = fwd
+    lib.moe_forward_prenorm.restype = I
+    lib.moe_forward_prenorm.argtypes = [SH, P, P, ctypes.c_float] + fwd[2:]
+    lib.moe_rmsnorm.restype = I
+    lib.moe_rmsnorm.argtypes = [SH, P, P, ctypes.c_float, P, P]
     lib.moe_route.restype = I
     lib.moe_route.argtypes = [SH, P, P, P, I, I, ctypes.c_float, P, P, P, SZ, P]
     lib.moe_permute.restype = I
@@ -201,6 +205,33 @@ def moe_forward(shape, x, W_router, expert_bias, W_gate, W_up, W_down, W_shared_
         _p(topk_w, torch.float32, (T, k), "topk_w"),
         _p(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream))
     _check(st, "moe_forward")
+
+
+def moe_forward_prenorm(shape, x, norm_gain, norm_eps, W_router, expert_bias, W_gate, W_up, W_down,
+                        W_shared_gate, W_shared_up, W_shared_down, score_fn, norm_topk, route_scale, out,
+                        topk_idx, topk_w, workspace, stream=None, W_shared_gate_vec=None):
+    """moe_forward behind the pre-norm RMSNorm (zero-centred gains): x is the raw
+    residual stream; the normalised rows are left in the workspace region "x_stage"."""
+    T, d, E, k = shape.T, shape.d_model, shape.E, shape.k
+    bf = torch.bfloat16
+    st = load().moe_forward_prenorm(
+        ctypes.byref(shape), _p(x, bf, (T, d), "x"), _p(norm_gain, bf, (d,), "norm_gain"), float(norm_eps),
+        _p(W_router, bf, (E, d), "W_router"), _p(expert_bias, torch.float32, (E,), "expert_bias"),
+        *_weights(shape, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down),
+        _gate_vec(shape, W_shared_gate_vec), _score(score_fn), int(bool(norm_topk)), float(route_scale),
+        _p(out, bf, (T, d), "out"), _p(topk_idx, torch.int32, (T, k), "topk_idx"),
+        _p(topk_w, torch.float32, (T, k), "topk_w"),
+        _p(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "moe_forward_prenorm")
+
+
+def moe_rmsnorm(shape, x, norm_gain, eps, x_norm, stream=None):
+    """x_norm = bf16(x / sqrt(mean(x^2) + eps) * (1 + norm_gain)), computed in double."""
+    T, d = shape.T, shape.d_model
+    bf = torch.bfloat16
+    st = load().moe_rmsnorm(ctypes.byref(shape), _p(x, bf, (T, d), "x"), _p(norm_gain, bf, (d,), "norm_gain"),
+                            float(eps), _p(x_norm, bf, (T, d), "x_norm"), _stream(stream))
+    _check(st, "moe_rmsnorm")
 
 
 def moe_forward_host(shape, x_host, W_router, expert_bias, W_gate, W_up, W_down, W_shared_gate,
@@ -339,6 +370,13 @@ class MoELayer:
 
     def __call__(self, x=None, stream=None):
         t, c = self.t, self.cfg
+        if c.prenorm:
+            moe_forward_prenorm(self.shape, t["x"] if x is None else x, t["norm_gain"], c.norm_eps, t["W_router"],
+                                t["expert_bias"], t["W_gate"], t["W_up"], t["W_down"], t["W_shared_gate"],
+                                t["W_shared_up"], t["W_shared_down"], c.score_fn, c.norm_topk, c.route_scale,
+                                self.out, self.topk_idx, self.topk_w, self.workspace, stream,
+                                W_shared_gate_vec=t.get("W_shared_gate_vec"))
+            return self.out, self.topk_idx, self.topk_w
         moe_forward(self.shape, t["x"] if x is None else x, t["W_router"], t["expert_bias"],
                     t["W_gate"], t["W_up"], t["W_down"], t["W_shared_gate"], t["W_shared_up"],
                     t["W_shared_down"], c.score_fn, c.norm_topk, c.route_scale, self.out,
@@ -353,16 +391,20 @@ class MoELayer:
         st = stream
         rec = (lambda i: events[i].record(st)) if events is not None else (lambda i: None)
         rec(0)
-        moe_route(s, t["x"], t["W_router"], t["expert_bias"], c.score_fn, c.norm_topk, c.route_scale,
+        x = t["x"]
+        if c.prenorm:
+            x = workspace_view(self.workspace, s, "x_stage", torch.bfloat16, (c.T, c.d))
+            moe_rmsnorm(s, t["x"], t["norm_gain"], c.norm_eps, x, st)
+        moe_route(s, x, t["W_router"], t["expert_bias"], c.score_fn, c.norm_topk, c.route_scale,
                   self.topk_idx, self.topk_w, self.workspace, st)
         rec(1)
         moe_permute(s, self.topk_idx, self.topk_w, self.workspace, st)
         rec(2)
-        moe_expert_gate_up(s, t["x"], t["W_gate"], t["W_up"], t["W_shared_gate"], t["W_shared_up"],
+        moe_expert_gate_up(s, x, t["W_gate"], t["W_up"], t["W_shared_gate"], t["W_shared_up"],
                            self.workspace, st)
         rec(3)
         moe_expert_down(s, t["W_down"], t["W_shared_down"], self.workspace, st)
         rec(4)
-        moe_combine(s, self.out, self.workspace, st, x=t["x"], W_shared_gate_vec=t.get("W_shared_gate_vec"))
+        moe_combine(s, self.out, self.workspace, st, x=x, W_shared_gate_vec=t.get("W_shared_gate_vec"))
         rec(5)
         return self.out, self.topk_idx, self.topk_w

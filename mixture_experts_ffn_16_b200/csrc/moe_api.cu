@@ -540,6 +540,49 @@ int moe_forward_host(const moe_shape* shape, const void* x_host, const void* W_r
   return MOE_OK;
 }
 
+int moe_rmsnorm(const moe_shape* shape, const void* x, const void* norm_gain, float eps, void* x_norm,
+                moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if (!x || !norm_gain || !x_norm || !(eps >= 0.0f) || !std::isfinite(eps)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(norm_gain) || !aligned16(x_norm)) return MOE_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return launch_rmsnorm(p, x, norm_gain, eps, x_norm, as_stream(stream));
+}
+
+int moe_forward_prenorm(const moe_shape* shape, const void* x, const void* norm_gain, float norm_eps,
+                        const void* W_router, const float* expert_bias, const void* W_gate, const void* W_up,
+                        const void* W_down, const void* W_shared_gate, const void* W_shared_up,
+                        const void* W_shared_down, const void* W_shared_gate_vec, int score_fn, int norm_topk,
+                        float route_scale, void* out, int32_t* topk_idx, float* topk_w, void* workspace,
+                        size_t workspace_bytes, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if (!norm_gain || !(norm_eps >= 0.0f) || !std::isfinite(norm_eps)) return MOE_ERR_INVALID_ARG;
+  if ((rc = check_route_args(x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w)) != MOE_OK)
+    return rc;
+  if (!aligned16(norm_gain)) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_expert_args(p, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down)) != MOE_OK)
+    return rc;
+  if (!out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out)) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_gate_vec(p, W_shared_gate_vec)) != MOE_OK) return rc;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = as_stream(stream);
+  void* xn = ws + p.xstage;
+  if ((rc = launch_rmsnorm(p, x, norm_gain, norm_eps, xn, st)) != MOE_OK) return rc;
+  // the shared-expert gate reads the block's input, i.e. the normalised rows
+  return forward_impl(p, di, xn, W_router, expert_bias, W_gate, W_up, W_down, W_shared_gate, W_shared_up,
+                      W_shared_down, W_shared_gate_vec, score_fn, norm_topk, route_scale, out, topk_idx, topk_w, ws,
+                      st);
+}
+
 int moe_workspace_region(const moe_shape* shape, int region, size_t* offset, size_t* bytes) {
   Plan p;
   if (!offset || !bytes) return MOE_ERR_INVALID_ARG;
@@ -556,6 +599,7 @@ int moe_workspace_region(const moe_shape* shape, int region, size_t* offset, siz
     case MOE_WS_H_SHARED: *offset = p.Hs; *bytes = S * Tp * p.fs * 2; break;
     case MOE_WS_Y: *offset = p.Yr; *bytes = R * p.d * 2; break;
     case MOE_WS_Y_SHARED: *offset = p.Ys; *bytes = S * Tp * p.d * 2; break;
+    case MOE_WS_X_STAGE: *offset = p.xstage; *bytes = T * p.d * 2; break;
     default: return MOE_ERR_INVALID_ARG;
   }
   return MOE_OK;

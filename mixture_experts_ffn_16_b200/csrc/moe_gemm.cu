@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  chain_wait();
   const int num_units = (MODE == kModeRouter) ? p.num_units_host : *p.num_units_dev;
 
   if (warp == 0) {
@@ -635,6 +636,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
   cluster_sync();                                    // peer barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  chain_wait();
   const int num_units = *p.num_units_dev;
   const uint32_t full_leader = mapa_shared(smem_u32(full), 0);     // + 8 * stage
   const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0); // + 8 * buf
@@ -954,8 +956,9 @@ static int launch_pair_mode(const GemmParams& prm, int grid, size_t smem, cudaSt
       return MOE_ERR_CUDA;
     configured[dev] = static_cast<int>(smem);
   }
-  moe_gemm_pair_kernel<MODE><<<grid, threads_of(MODE), smem, st>>>(prm);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_chained(moe_gemm_pair_kernel<MODE>, dim3(grid), dim3(threads_of(MODE)), smem, st, prm) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 int launch_gemm_pair(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st) {
@@ -980,8 +983,9 @@ static int launch_mode(const GemmParams& prm, int grid, size_t smem, cudaStream_
       return MOE_ERR_CUDA;
     configured[dev] = static_cast<int>(smem);
   }
-  moe_gemm_kernel<MODE><<<grid, threads_of(MODE), smem, st>>>(prm);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_chained(moe_gemm_kernel<MODE>, dim3(grid), dim3(threads_of(MODE)), smem, st, prm) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st) {

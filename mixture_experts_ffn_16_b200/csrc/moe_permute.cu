@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(kPermBlock)
 permute_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
                      int32_t* __restrict__ blkcnt, uint32_t* err) {
   extern __shared__ uint32_t masks[];
+  chain_wait();
   build_masks(topk_idx, T, E, k, masks, err);
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int c = 0;
@@ -126,6 +127,7 @@ struct ScanArgs {
 };
 
 __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) {
+  chain_wait();
   // Experts per thread: E <= 2048 -> at most 2.
   constexpr int kPer = (kMaxE + kScanThreads - 1) / kScanThreads;
   int cnt[kPer], pad[kPer], u1[kPer], u2[kPer];
@@ -216,6 +218,7 @@ permute_scatter_kernel(const int32_t* __restrict__ topk_idx, const float* __rest
                        int32_t* __restrict__ perm, float* __restrict__ roww, int32_t* __restrict__ inv,
                        uint32_t* err) {
   extern __shared__ uint32_t masks[];
+  chain_wait();
   build_masks(topk_idx, T, E, k, masks, err);
   const int t = blockIdx.x * kPermBlock + threadIdx.x;
   if (t >= T) return;
@@ -254,8 +257,9 @@ int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, 
       return MOE_ERR_CUDA;
     configured[dev] = 1;
   }
-  permute_count_kernel<<<p.nb, kPermBlock, msmem, st>>>(topk_idx, p.T, p.E, p.k, blkcnt, err);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_chained(permute_count_kernel, dim3(p.nb), dim3(kPermBlock), msmem, st, topk_idx, p.T, p.E, p.k, blkcnt,
+                     err) != cudaSuccess)
+    return MOE_ERR_CUDA;
 
   ScanArgs a;
   a.blkcnt = blkcnt;
@@ -279,13 +283,13 @@ int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, 
   a.S = p.S;
   a.shared_units1 = p.shared_units1;
   a.shared_units2 = p.shared_units2;
-  permute_scan_kernel<<<1, kScanThreads, 0, st>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_chained(permute_scan_kernel, dim3(1), dim3(kScanThreads), 0, st, a) != cudaSuccess) return MOE_ERR_CUDA;
 
-  permute_scatter_kernel<<<p.nb, kPermBlock, msmem, st>>>(
-      topk_idx, topk_w, p.T, p.E, p.k, blkcnt, a.roff, a.perm, a.roww,
-      reinterpret_cast<int32_t*>(ws + p.inv), err);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_chained(permute_scatter_kernel, dim3(p.nb), dim3(kPermBlock), msmem, st, topk_idx, topk_w, p.T, p.E,
+                        p.k, blkcnt, a.roff, a.perm, a.roww, reinterpret_cast<int32_t*>(ws + p.inv),
+                        err) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

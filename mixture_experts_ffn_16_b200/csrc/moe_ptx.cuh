@@ -391,4 +391,9 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- chained launch
+// Wait for the previous kernel in the stream (complete, writes visible); a
+// no-op for a kernel launched without programmatic serialisation.
+__device__ __forceinline__ void chain_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 }  // namespace moe

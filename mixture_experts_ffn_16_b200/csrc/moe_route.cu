@@ -16,6 +16,7 @@
 #include <cmath>
 
 #include "moe_internal.h"
+#include "moe_ptx.cuh"
 
 namespace moe {
 
@@ -39,6 +40,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
             int score_fn, int norm_topk, float route_scale, int32_t* __restrict__ topk_idx,
             float* __restrict__ topk_w) {
+  chain_wait();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -127,8 +129,10 @@ template <int NPL>
 int launch_npl(const float* logits, const float* bias, int T, int E, int k, int fn, int norm,
                float scale, int32_t* idx, float* w, cudaStream_t st) {
   const int grid = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  topk_kernel<NPL><<<grid, kWarpsPerBlock * 32, 0, st>>>(logits, bias, T, E, k, fn, norm, scale, idx, w);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_chained(topk_kernel<NPL>, dim3(grid), dim3(kWarpsPerBlock * 32), 0, st, logits, bias, T, E, k, fn,
+                        norm, scale, idx, w) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 }  // namespace

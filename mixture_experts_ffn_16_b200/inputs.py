@@ -8,8 +8,9 @@ Recipe (same for every workload):
     seed;
   * draw order: x, W_router, expert_bias, W_gate, W_up, W_down,
     W_shared_gate, W_shared_up, W_shared_down, then (gated shared expert only)
-    W_shared_gate_vec [S,d], then (skewed workload only) the shuffled expert
-    ranks;
+    W_shared_gate_vec [S,d], then (pre-norm only) the zero-centred RMSNorm
+    gains norm_gain [d] ~ N(0, 0.1), then (skewed workload only) the shuffled
+    expert ranks;
   * each tensor is drawn as fp32 N(0, std) in slabs of at most 2**27 elements
     along its first axis, then rounded to bf16 (expert_bias stays fp32);
   * x ~ N(0, 1); all weights ~ N(0, 0.02); expert_bias ~ N(0, 0.1) where the
@@ -45,6 +46,8 @@ class MoEConfig:
     bias_std: float = 0.0              # 0 = no expert_bias tensor
     skew: str = ""                     # "" | "zipf_rank"
     shared_gate: bool = False          # per-token sigmoid gate on the shared experts (Qwen3.5)
+    prenorm: bool = False              # pre-norm RMSNorm (zero-centred gains) in front of the block
+    norm_eps: float = 1e-6
     seed: int = 0
     x_std: float = 1.0
     w_std: float = 0.02
@@ -113,6 +116,9 @@ def make_inputs(cfg: MoEConfig, device="cpu", seed=None):
     W_shared_gate_vec = None
     if cfg.shared_gate and S > 0:
         W_shared_gate_vec = _randn_bf16((S, d), cfg.w_std, gen, device)
+    norm_gain = None
+    if cfg.prenorm:
+        norm_gain = _randn_bf16((d,), 0.1, gen, device)
     ranks = None
     if cfg.skew == "zipf_rank":
         ranks = torch.randperm(E, generator=gen, device=device) + 1
@@ -121,7 +127,7 @@ def make_inputs(cfg: MoEConfig, device="cpu", seed=None):
         W_router[:, 0] = offset.to(torch.bfloat16)
     return dict(x=x, W_router=W_router, expert_bias=bias, W_gate=W_gate, W_up=W_up, W_down=W_down,
                 W_shared_gate=W_shared_gate, W_shared_up=W_shared_up, W_shared_down=W_shared_down,
-                W_shared_gate_vec=W_shared_gate_vec, ranks=ranks)
+                W_shared_gate_vec=W_shared_gate_vec, norm_gain=norm_gain, ranks=ranks)
 
 
 def bf16_bits(t):

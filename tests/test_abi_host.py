@@ -151,3 +151,32 @@ def test_experts_forward_argument_checks(lib):
     assert call(shape=s0, weights=w6[:3] + [None] * 3, gv=P(4096),
                 ws_bytes=api.moe_workspace_bytes(s0)) == api.MOE_ERR_INVALID_ARG
     assert call(ws_bytes=n - 1) == api.MOE_ERR_WORKSPACE
+
+
+def test_prenorm_and_rmsnorm_argument_checks(lib):
+    s = api.make_shape(16, 128, 8, 2, 128, 1, 128)
+    n = api.moe_workspace_bytes(s)
+    P = ctypes.c_void_p
+    good = [P(4096)] * 9
+
+    def fwd(gain=P(4096), eps=1e-6, x=P(4096)):
+        return lib.moe_forward_prenorm(ctypes.byref(s), x, gain, eps, *good[1:], None, 0, 1, 1.0,
+                                       P(4096), P(4096), P(4096), P(4096), n, None)
+
+    assert fwd(gain=None) == api.MOE_ERR_INVALID_ARG
+    assert fwd(eps=-1.0) == api.MOE_ERR_INVALID_ARG
+    assert fwd(eps=float("nan")) == api.MOE_ERR_INVALID_ARG
+    assert fwd(eps=float("inf")) == api.MOE_ERR_INVALID_ARG
+    assert fwd(x=None) == api.MOE_ERR_INVALID_ARG
+    assert fwd(gain=P(4098)) == api.MOE_ERR_UNSUPPORTED
+    assert lib.moe_rmsnorm(ctypes.byref(s), P(4096), None, 1e-6, P(4096), None) == api.MOE_ERR_INVALID_ARG
+    assert lib.moe_rmsnorm(ctypes.byref(s), P(4096), P(4096), -1.0, P(4096), None) == api.MOE_ERR_INVALID_ARG
+    assert lib.moe_rmsnorm(ctypes.byref(s), P(4096), P(4096), 1e-6, P(4100), None) == api.MOE_ERR_UNSUPPORTED
+    bad = api.make_shape(16, 100, 8, 2, 128, 1, 128)
+    assert lib.moe_rmsnorm(ctypes.byref(bad), P(4096), P(4096), 1e-6, P(4096), None) == api.MOE_ERR_UNSUPPORTED
+
+
+def test_x_stage_region(lib):
+    s = api.make_shape(16, 128, 8, 2, 128, 1, 128)
+    off, nb = api.moe_workspace_region(s, "x_stage")
+    assert nb == 16 * 128 * 2 and off % 256 == 0 and off + nb <= api.moe_workspace_bytes(s)

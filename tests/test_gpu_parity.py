@@ -174,3 +174,72 @@ def test_external_routing_matches_oracle(oracle_mod, cfg):
     err = np.abs(got - ref["out"]).max()
     print(cfg.name, "external routing err ratio", err / scale)
     assert np.isfinite(got).all() and err <= 2e-2 * scale
+
+
+# ---------------------------------------------------------------- pre-norm RMSNorm prologue
+
+def _x_norm_oracle(oracle_mod, inp, cfg):
+    from mixture_experts_ffn_16_b200.inputs import bf16_bits
+    eps = float(np.float32(cfg.norm_eps))         # the ABI takes eps as binary32
+    return oracle_mod.rmsnorm(bf16_bits(inp["x"]), bf16_bits(inp["norm_gain"]), eps)["y_bits"]
+
+
+@pytest.mark.parametrize("T,d,x_std", [(300, 512, 3.0), (17, 7168, 0.05), (5, 64, 1.0), (1000, 2048, 40.0)])
+def test_rmsnorm_bit_exact(oracle_mod, T, d, x_std):
+    """x_norm is computed in double and rounded once, so it matches the oracle's
+    double-precision definition bit for bit, including a zero row."""
+    _need_gpu()
+    from mixture_experts_ffn_16_b200.inputs import bf16_bits
+    cfg = MoEConfig("rmsnorm_only", T=T, d=d, E=4, k=1, f=64, S=0, fs=0, x_std=x_std, prenorm=True, seed=30)
+    inp = make_inputs(cfg, device="cuda")
+    inp["x"][T // 2].zero_()
+    shape = api.shape_of(cfg)
+    y = torch.empty_like(inp["x"])
+    api.moe_rmsnorm(shape, inp["x"], inp["norm_gain"], cfg.norm_eps, y)
+    ref = _x_norm_oracle(oracle_mod, inp, cfg)
+    got = bf16_bits(y)
+    assert not got[T // 2].any()
+    assert np.array_equal(got, ref), f"{int((got != ref).sum())} of {got.size} values differ"
+
+
+PRENORM = [
+    MoEConfig("prenorm_softmax", T=300, d=512, E=40, k=6, f=192, S=1, fs=320, prenorm=True, x_std=4.0, seed=31),
+    MoEConfig("prenorm_gated_qwen_like", T=200, d=256, E=64, k=10, f=64, S=1, fs=128, prenorm=True,
+              shared_gate=True, x_std=0.3, seed=32),
+    MoEConfig("prenorm_sigmoid_bias", T=129, d=384, E=24, k=4, f=128, S=2, fs=64, prenorm=True,
+              score_fn="sigmoid", bias_std=0.1, x_std=10.0, seed=33),
+]
+
+
+@pytest.mark.parametrize("cfg", PRENORM, ids=lambda c: c.name)
+def test_prenorm_block_every_token(oracle_mod, cfg):
+    """moe_forward_prenorm: the staged rows equal the oracle's RMSNorm exactly,
+    and the block on them matches the oracle's block on the oracle's rows."""
+    _need_gpu()
+    inp = make_inputs(cfg, device="cuda")
+    out, idx, w, layer = run_gpu(cfg, inp)
+    xn = api.workspace_view(layer.workspace, layer.shape, "x_stage", torch.bfloat16, (cfg.T, cfg.d))
+    from mixture_experts_ffn_16_b200.inputs import bf16_bits
+    ref_xn = _x_norm_oracle(oracle_mod, inp, cfg)
+    assert np.array_equal(bf16_bits(xn), ref_xn)
+    host = oracle_args(inp)
+    host["x"] = ref_xn
+    rep = check_parity(oracle_mod, cfg, host, out, idx, w)
+    print(cfg.name, rep)
+
+
+def test_prenorm_full_size_sampled(oracle_mod):
+    cfg = MoEConfig("prefill_softmax_prenorm", T=4096, d=2048, E=256, k=8, f=512, S=1, fs=512, prenorm=True,
+                    x_std=2.0, seed=34)
+    _need_gpu()
+    inp = make_inputs(cfg, device="cuda")
+    out, idx, w, layer = run_gpu(cfg, inp)
+    xn = api.workspace_view(layer.workspace, layer.shape, "x_stage", torch.bfloat16, (cfg.T, cfg.d))
+    from mixture_experts_ffn_16_b200.inputs import bf16_bits
+    ref_xn = _x_norm_oracle(oracle_mod, inp, cfg)
+    assert np.array_equal(bf16_bits(xn), ref_xn)
+    tokens = _sample(cfg.T, 192, seed=35)
+    host = oracle_args(inp)
+    host["x"] = ref_xn
+    rep = check_parity(oracle_mod, cfg, host, out[tokens], idx[tokens], w[tokens], tokens=tokens)
+    print(cfg.name, rep)
