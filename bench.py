@@ -34,7 +34,7 @@ if ROOT not in sys.path:
 
 from mixture_experts_ffn_16_b200 import api  # noqa: E402
 from mixture_experts_ffn_16_b200.inputs import CONFIGS, make_inputs, oracle_args  # noqa: E402
-from mixture_experts_ffn_16_b200.roofline import (block_cost, kernel_costs, measured_peaks,  # noqa: E402
+from mixture_experts_ffn_16_b200.roofline import (block_cost, kernel_costs, measured_peaks, weight_bytes,  # noqa: E402
                                                   measured_traffic)
 
 METRIC = "MoE-layer tokens/sec at 1 B200; % bf16 tensor peak (prefill) / % HBM BW (decode)"
@@ -56,10 +56,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--variant", default="", choices=["", "gated_shared", "external_routing", "prenorm"],
+    ap.add_argument("--variant", default="", choices=["", "gated_shared", "external_routing", "prenorm", "fp8"],
                     help="gated_shared: Qwen3.5-style sigmoid gate on the shared experts; "
                          "external_routing: routing supplied by the caller (steps a3..a7 only); "
-                         "prenorm: the pre-norm RMSNorm (zero-centred gains) fused in front")
+                         "prenorm: the pre-norm RMSNorm (zero-centred gains) fused in front; "
+                         "fp8: block-scaled FP8 expert weights")
     return ap.parse_args()
 
 
@@ -257,11 +258,18 @@ def run_ours(args, cfg):
                         layer.workspace, stream)
         if ev is not None:
             ev[2].record(stream)
-        api.moe_expert_gate_up(s, xb, t["W_gate"], t["W_up"], t["W_shared_gate"], t["W_shared_up"],
-                               layer.workspace, stream)
+        if c.fp8:
+            api.moe_expert_gate_up_fp8(s, xb, t["W_gate_f8"], t["W_up_f8"], t["W_shared_gate_f8"],
+                                       t["W_shared_up_f8"], layer.workspace, stream)
+        else:
+            api.moe_expert_gate_up(s, xb, t["W_gate"], t["W_up"], t["W_shared_gate"], t["W_shared_up"],
+                                   layer.workspace, stream)
         if ev is not None:
             ev[3].record(stream)
-        api.moe_expert_down(s, t["W_down"], t["W_shared_down"], layer.workspace, stream)
+        if c.fp8:
+            api.moe_expert_down_fp8(s, t["W_down_f8"], t["W_shared_down_f8"], layer.workspace, stream)
+        else:
+            api.moe_expert_down(s, t["W_down"], t["W_shared_down"], layer.workspace, stream)
         if ev is not None:
             ev[4].record(stream)
         api.moe_combine(s, layer.out, layer.workspace, stream, x=xb,
@@ -305,9 +313,10 @@ def run_ours(args, cfg):
     # still copies its x in and its out / topk_idx / topk_w back inside the
     # timed region.
     e2e = None
-    # the host-buffer entry point runs the whole block on raw x: it has no
-    # caller-routing or pre-norm form, so those variants report no e2e figure
-    if not args.no_e2e and not external and not cfg.prenorm:
+    # the host-buffer entry point runs the whole block on raw x with bf16
+    # weights: it has no caller-routing, pre-norm or FP8 form, so those
+    # variants report no e2e figure
+    if not args.no_e2e and not external and not cfg.prenorm and not cfg.fp8:
         lanes = []
         NL = 3
         for li in range(NL):
@@ -393,8 +402,9 @@ def run_ours(args, cfg):
                            "d_ff": cfg.f, "n_shared": cfg.S, "d_ff_shared": cfg.fs, "score_fn": cfg.score_fn,
                            "norm_topk": cfg.norm_topk, "touched_experts": touched,
                            "variant": args.variant or "base",
+                           "expert_weights": "fp8 e4m3 + ue8m0 scale per 32" if cfg.fp8 else "bf16",
                            "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (
-                               2.0 * cfg.E * 3 * cfg.f * cfg.d / 1e9),
+                               weight_bytes(cfg) * cfg.E * 3 * cfg.f * cfg.d / 1e9),
                            "parallelism": "replicas" if world > 1 else "single GPU"},
                 "roofline": roof, "step_roofline": step_roof,
                 "kernels_us": stage_avg_us, "cpu_baseline": cpu, "e2e": e2e,
@@ -416,6 +426,8 @@ def main():
         cfg = dataclasses.replace(cfg, shared_gate=True)
     if args.variant == "prenorm":
         cfg = dataclasses.replace(cfg, prenorm=True)
+    if args.variant == "fp8":
+        cfg = dataclasses.replace(cfg, fp8=True)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

@@ -165,6 +165,49 @@ MOE_API int moe_forward_prenorm(const moe_shape *shape,
 MOE_API int moe_rmsnorm(const moe_shape *shape, const void *x, const void *norm_gain, float eps,
                 void *x_norm, moe_stream_t stream);
 
+/* ---- Block-scaled FP8 expert weights ----
+ * The pages name an official FP8 weight release and "block-scaled FP8"
+ * (qwen3-5-vs-gemma-4, component table, Qwen3.5 routed-experts cell;
+ * qwen3-5-vs-deepseek-v4, blueprint diagram) but give no block size or scale
+ * format.  Reading: OCP MX-style blocks of 32 consecutive elements along the
+ * input dimension K, one power-of-two scale per block stored as its biased
+ * exponent byte (UE8M0).  Element [g, r, c] of the weight is
+ *     e4m3(codes[g, r, c]) * 2^(scales[g, c / 32, r] - 127)
+ * with codes in the [out, in] layout of the bf16 weight and the scales
+ * block-major.  E4M3 is the OCP "E4M3FN" encoding (no infinities, 0x7F/0xFF
+ * NaN).  The library widens each tile to bf16 in shared memory; the widened
+ * value is exact whenever it is representable in bf16 (scale bytes 10..246
+ * for finite codes), so the block then computes exactly what moe_forward
+ * computes on the widened weights, while HBM moves half the weight bytes. */
+typedef struct {
+  const void *codes;    /* uint8 E4M3 [G, rows, K], 16-byte aligned */
+  const void *scales;   /* uint8 UE8M0 [G, K/32, rows], 16-byte aligned */
+} moe_fp8_weight;
+
+/* moe_forward with FP8 routed and shared expert weights (W_router stays
+ * bf16).  W_gate / W_up: G = E, rows = d_ff, K = d_model; W_down: G = E,
+ * rows = d_model, K = d_ff; shared: G = n_shared with d_ff_shared.  The
+ * shared pointers are NULL iff n_shared == 0; a moe_fp8_weight with a NULL
+ * member is MOE_ERR_INVALID_ARG.  Everything else as in moe_forward. */
+MOE_API int moe_forward_fp8(const moe_shape *shape,
+                const void *x, const void *W_router, const float *expert_bias,
+                const moe_fp8_weight *W_gate, const moe_fp8_weight *W_up, const moe_fp8_weight *W_down,
+                const moe_fp8_weight *W_shared_gate, const moe_fp8_weight *W_shared_up,
+                const moe_fp8_weight *W_shared_down, const void *W_shared_gate_vec,
+                int score_fn, int norm_topk, float route_scale,
+                void *out, int32_t *topk_idx, float *topk_w,
+                void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* The FP8 forms of the two expert steps (a4 + a6, a5 + a6), for callers that
+ * run the steps one by one. */
+MOE_API int moe_expert_gate_up_fp8(const moe_shape *shape, const void *x, const moe_fp8_weight *W_gate,
+                const moe_fp8_weight *W_up, const moe_fp8_weight *W_shared_gate,
+                const moe_fp8_weight *W_shared_up, void *workspace, size_t workspace_bytes,
+                moe_stream_t stream);
+MOE_API int moe_expert_down_fp8(const moe_shape *shape, const moe_fp8_weight *W_down,
+                const moe_fp8_weight *W_shared_down, void *workspace, size_t workspace_bytes,
+                moe_stream_t stream);
+
 /* ---- The steps of moe_forward, callable one by one (same arguments and
  * rules; each step reads what the previous steps left in the workspace, so
  * they must be called in this order with the same shape and workspace). ---- */

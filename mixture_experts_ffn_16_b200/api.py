@@ -32,7 +32,8 @@ WS_REGIONS = {"logits": 0, "counts": 1, "offsets": 2, "perm": 3, "row_w": 4, "in
 EXPORTED = ["moe_version", "moe_status_string", "moe_workspace_bytes", "moe_forward",
             "moe_forward_host", "moe_route", "moe_permute", "moe_expert_gate_up", "moe_expert_down",
             "moe_combine", "moe_workspace_region", "moe_device_status", "moe_debug_wait_timeout",
-            "moe_route_noalloc", "moe_experts_forward", "moe_rmsnorm", "moe_forward_prenorm"]
+            "moe_route_noalloc", "moe_experts_forward", "moe_rmsnorm", "moe_forward_prenorm",
+            "moe_forward_fp8", "moe_expert_gate_up_fp8", "moe_expert_down_fp8"]
 
 
 class MoEError(RuntimeError):
@@ -45,6 +46,11 @@ class MoeShape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d_model", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("n_shared", ctypes.c_int32),
                 ("d_ff_shared", ctypes.c_int32)]
+
+
+class MoeFp8Weight(ctypes.Structure):
+    """moe_fp8_weight: E4M3 codes [G, rows, K] and UE8M0 block scales [G, K/32, rows]."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
 _lib = None
@@ -74,6 +80,13 @@ def load():
     lib.moe_forward_host.argtypes = fwd
     lib.moe_forward_prenorm.restype = I
     lib.moe_forward_prenorm.argtypes = [SH, P, P, ctypes.c_float] + fwd[2:]
+    F8 = ctypes.POINTER(MoeFp8Weight)
+    lib.moe_forward_fp8.restype = I
+    lib.moe_forward_fp8.argtypes = [SH, P, P, P, F8, F8, F8, F8, F8, F8] + fwd[10:]
+    lib.moe_expert_gate_up_fp8.restype = I
+    lib.moe_expert_gate_up_fp8.argtypes = [SH, P, F8, F8, F8, F8, P, SZ, P]
+    lib.moe_expert_down_fp8.restype = I
+    lib.moe_expert_down_fp8.argtypes = [SH, F8, F8, P, SZ, P]
     lib.moe_rmsnorm.restype = I
     lib.moe_rmsnorm.argtypes = [SH, P, P, ctypes.c_float, P, P]
     lib.moe_route.restype = I
@@ -185,6 +198,24 @@ def _weights(shape, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_d
             _p(W_shared_down, bf, (S, d, fs), "W_shared_down") if S else None]
 
 
+def _f8(w, G, rows, K, name):
+    """(codes, scales) tensors -> a MoeFp8Weight (None when w is None)."""
+    if w is None:
+        return None
+    codes, scales = w
+    return MoeFp8Weight(_p(codes, torch.uint8, (G, rows, K), name + ".codes"),
+                        _p(scales, torch.uint8, (G, K // 32, rows), name + ".scales"))
+
+
+def _f8_weights(shape, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down):
+    E, f, d, S, fs = shape.E, shape.d_ff, shape.d_model, shape.n_shared, shape.d_ff_shared
+    ws = [_f8(W_gate, E, f, d, "W_gate"), _f8(W_up, E, f, d, "W_up"), _f8(W_down, E, d, f, "W_down"),
+          _f8(W_shared_gate, S, fs, d, "W_shared_gate") if S else None,
+          _f8(W_shared_up, S, fs, d, "W_shared_up") if S else None,
+          _f8(W_shared_down, S, d, fs, "W_shared_down") if S else None]
+    return [None if w is None else ctypes.pointer(w) for w in ws]
+
+
 def _gate_vec(shape, W_shared_gate_vec):
     if W_shared_gate_vec is None:
         return None
@@ -223,6 +254,40 @@ def moe_forward_prenorm(shape, x, norm_gain, norm_eps, W_router, expert_bias, W_
         _p(topk_w, torch.float32, (T, k), "topk_w"),
         _p(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream))
     _check(st, "moe_forward_prenorm")
+
+
+def moe_forward_fp8(shape, x, W_router, expert_bias, W_gate, W_up, W_down, W_shared_gate, W_shared_up,
+                    W_shared_down, score_fn, norm_topk, route_scale, out, topk_idx, topk_w, workspace,
+                    stream=None, W_shared_gate_vec=None):
+    """moe_forward with block-scaled FP8 expert weights: each W_* is a
+    (codes uint8 [G, rows, K], scales uint8 [G, K/32, rows]) pair, or None for
+    the shared ones when n_shared == 0."""
+    T, d, E, k = shape.T, shape.d_model, shape.E, shape.k
+    bf = torch.bfloat16
+    st = load().moe_forward_fp8(
+        ctypes.byref(shape), _p(x, bf, (T, d), "x"), _p(W_router, bf, (E, d), "W_router"),
+        _p(expert_bias, torch.float32, (E,), "expert_bias"),
+        *_f8_weights(shape, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down),
+        _gate_vec(shape, W_shared_gate_vec), _score(score_fn), int(bool(norm_topk)), float(route_scale),
+        _p(out, bf, (T, d), "out"), _p(topk_idx, torch.int32, (T, k), "topk_idx"),
+        _p(topk_w, torch.float32, (T, k), "topk_w"),
+        _p(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "moe_forward_fp8")
+
+
+def moe_expert_gate_up_fp8(shape, x, W_gate, W_up, W_shared_gate, W_shared_up, workspace, stream=None):
+    w = _f8_weights(shape, W_gate, W_up, None, W_shared_gate, W_shared_up, None)
+    st = load().moe_expert_gate_up_fp8(ctypes.byref(shape), _p(x, torch.bfloat16, (shape.T, shape.d_model), "x"),
+                                       w[0], w[1], w[3], w[4], _p(workspace, torch.uint8, None, "workspace"),
+                                       workspace.numel(), _stream(stream))
+    _check(st, "moe_expert_gate_up_fp8")
+
+
+def moe_expert_down_fp8(shape, W_down, W_shared_down, workspace, stream=None):
+    w = _f8_weights(shape, None, None, W_down, None, None, W_shared_down)
+    st = load().moe_expert_down_fp8(ctypes.byref(shape), w[2], w[5], _p(workspace, torch.uint8, None, "workspace"),
+                                    workspace.numel(), _stream(stream))
+    _check(st, "moe_expert_down_fp8")
 
 
 def moe_rmsnorm(shape, x, norm_gain, eps, x_norm, stream=None):
@@ -367,9 +432,18 @@ class MoELayer:
         self.out = torch.empty((T, d), dtype=torch.bfloat16, device=device)
         self.topk_idx = torch.empty((T, k), dtype=torch.int32, device=device)
         self.topk_w = torch.empty((T, k), dtype=torch.float32, device=device)
+        if cfg.fp8 and cfg.prenorm:
+            raise ValueError("MoELayer: the FP8 and pre-norm forms are separate entry points")
 
     def __call__(self, x=None, stream=None):
         t, c = self.t, self.cfg
+        if c.fp8:
+            moe_forward_fp8(self.shape, t["x"] if x is None else x, t["W_router"], t["expert_bias"],
+                            t["W_gate_f8"], t["W_up_f8"], t["W_down_f8"], t["W_shared_gate_f8"],
+                            t["W_shared_up_f8"], t["W_shared_down_f8"], c.score_fn, c.norm_topk, c.route_scale,
+                            self.out, self.topk_idx, self.topk_w, self.workspace, stream,
+                            W_shared_gate_vec=t.get("W_shared_gate_vec"))
+            return self.out, self.topk_idx, self.topk_w
         if c.prenorm:
             moe_forward_prenorm(self.shape, t["x"] if x is None else x, t["norm_gain"], c.norm_eps, t["W_router"],
                                 t["expert_bias"], t["W_gate"], t["W_up"], t["W_down"], t["W_shared_gate"],
@@ -400,10 +474,17 @@ class MoELayer:
         rec(1)
         moe_permute(s, self.topk_idx, self.topk_w, self.workspace, st)
         rec(2)
-        moe_expert_gate_up(s, x, t["W_gate"], t["W_up"], t["W_shared_gate"], t["W_shared_up"],
-                           self.workspace, st)
+        if c.fp8:
+            moe_expert_gate_up_fp8(s, x, t["W_gate_f8"], t["W_up_f8"], t["W_shared_gate_f8"],
+                                   t["W_shared_up_f8"], self.workspace, st)
+        else:
+            moe_expert_gate_up(s, x, t["W_gate"], t["W_up"], t["W_shared_gate"], t["W_shared_up"],
+                               self.workspace, st)
         rec(3)
-        moe_expert_down(s, t["W_down"], t["W_shared_down"], self.workspace, st)
+        if c.fp8:
+            moe_expert_down_fp8(s, t["W_down_f8"], t["W_shared_down_f8"], self.workspace, st)
+        else:
+            moe_expert_down(s, t["W_down"], t["W_shared_down"], self.workspace, st)
         rec(4)
         moe_combine(s, self.out, self.workspace, st, x=x, W_shared_gate_vec=t.get("W_shared_gate_vec"))
         rec(5)

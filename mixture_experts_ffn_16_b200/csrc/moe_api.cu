@@ -48,6 +48,48 @@ bool map_weights(CUtensorMap* m, const void* ptr, int K, int rows, int G) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Block-scaled FP8 weight: codes [G, rows, K] uint8 -> tiles of 128 rows x 64
+// codes (unswizzled 64-byte rows); scales [G, K/32, rows] uint8 -> tiles of
+// 128 rows x 2 blocks.
+bool map_f8_codes(CUtensorMap* m, const void* ptr, int K, int rows, int G) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(G)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(K) * rows};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(kTileRows), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool map_f8_scales(CUtensorMap* m, const void* ptr, int K, int rows, int G) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const int nb = K / 32;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(G)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(rows) * nb};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kTileRows), static_cast<cuuint32_t>(kTileK / 32), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// An expert weight operand: bf16 (s == nullptr), or block-scaled FP8 codes
+// (p) with their scales (s).
+struct Wt {
+  const void* p = nullptr;
+  const void* s = nullptr;
+  Wt(const void* d = nullptr) : p(d) {}   // NOLINT: bf16 pointers convert implicitly
+  Wt(const void* d, const void* sc) : p(d), s(sc) {}
+};
+
+bool map_weight_operand(CUtensorMap* a, CUtensorMap* sc, const Wt& w, int K, int rows, int G) {
+  if (w.s) return map_f8_codes(a, w.p, K, rows, G) && map_f8_scales(sc, w.s, K, rows, G);
+  return map_weights(a, w.p, K, rows, G);
+}
+
 // Token-row source [rows, K] bf16, 128-byte swizzle, box of box_rows rows.
 bool map_rows(CUtensorMap* m, const void* ptr, int K, int rows, int box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -121,19 +163,23 @@ int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_
                      route_scale, topk_idx, topk_w, st);
 }
 
-int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* Wg, const void* Wu,
-                const void* Wsg, const void* Wsu, char* ws, cudaStream_t st) {
+int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, Wt Wg, Wt Wu, Wt Wsg, Wt Wsu, char* ws,
+                cudaStream_t st) {
   GemmParams g;
   std::memset(&g, 0, sizeof g);
-  if (!map_weights(&g.mapA[0], Wg, p.d, p.f, p.E) || !map_weights(&g.mapA[1], Wu, p.d, p.f, p.E) ||
-      !map_rows_set(g.mapB[0], x, p.d, p.T))
+  const bool f8 = Wg.s != nullptr;
+  if (!map_weight_operand(&g.mapA[0], &g.mapS[0], Wg, p.d, p.f, p.E) ||
+      !map_weight_operand(&g.mapA[1], &g.mapS[1], Wu, p.d, p.f, p.E) || !map_rows_set(g.mapB[0], x, p.d, p.T))
     return MOE_ERR_CUDA;
   if (p.S > 0) {
-    if (!map_weights(&g.mapA[2], Wsg, p.d, p.fs, p.S) || !map_weights(&g.mapA[3], Wsu, p.d, p.fs, p.S))
+    if (!map_weight_operand(&g.mapA[2], &g.mapS[2], Wsg, p.d, p.fs, p.S) ||
+        !map_weight_operand(&g.mapA[3], &g.mapS[3], Wsu, p.d, p.fs, p.S))
       return MOE_ERR_CUDA;
   } else {
     g.mapA[2] = g.mapA[0];
     g.mapA[3] = g.mapA[1];
+    g.mapS[2] = g.mapS[0];
+    g.mapS[3] = g.mapS[1];
   }
   copy_set(g.mapB[1], g.mapB[0]);
   g.units = reinterpret_cast<const int4*>(ws + p.units1);
@@ -149,6 +195,14 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* 
   g.weights_evict_first = p.weights_evict_first;
   int stages = 0;
   g.nbuf = (2 * p.nmax1 <= 256) ? 2 : 1;
+  if (f8) {
+    int raw = 0, tok = 0;
+    const size_t smem = gemm_f8_smem_bytes(kModeGateUp, p.nmax1, &stages, &tok, &raw);
+    g.stages = stages;
+    g.tok_stages = tok;
+    g.raw_stages = raw;
+    return launch_gemm(kModeGateUp, g, di.sms, smem, st, true);
+  }
   if (p.pair1) {
     const size_t smem = gemm_pair_smem_bytes(kModeGateUp, p.nmax1, &stages);
     g.stages = stages;
@@ -159,20 +213,26 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, const void* 
   return launch_gemm(kModeGateUp, g, di.sms, smem, st);
 }
 
-int run_down(const Plan& p, const DeviceInfo& di, const void* Wd, const void* Wsd, char* ws, cudaStream_t st) {
+int run_down(const Plan& p, const DeviceInfo& di, Wt Wd, Wt Wsd, char* ws, cudaStream_t st) {
   GemmParams g;
   std::memset(&g, 0, sizeof g);
-  if (!map_weights(&g.mapA[0], Wd, p.f, p.d, p.E) || !map_rows_set(g.mapB[0], ws + p.Hr, p.f, p.Rcap))
+  const bool f8 = Wd.s != nullptr;
+  if (!map_weight_operand(&g.mapA[0], &g.mapS[0], Wd, p.f, p.d, p.E) ||
+      !map_rows_set(g.mapB[0], ws + p.Hr, p.f, p.Rcap))
     return MOE_ERR_CUDA;
   if (p.S > 0) {
-    if (!map_weights(&g.mapA[2], Wsd, p.fs, p.d, p.S) || !map_rows_set(g.mapB[1], ws + p.Hs, p.fs, p.S * p.Tp))
+    if (!map_weight_operand(&g.mapA[2], &g.mapS[2], Wsd, p.fs, p.d, p.S) ||
+        !map_rows_set(g.mapB[1], ws + p.Hs, p.fs, p.S * p.Tp))
       return MOE_ERR_CUDA;
   } else {
     g.mapA[2] = g.mapA[0];
+    g.mapS[2] = g.mapS[0];
     copy_set(g.mapB[1], g.mapB[0]);
   }
   g.mapA[1] = g.mapA[0];
   g.mapA[3] = g.mapA[2];
+  g.mapS[1] = g.mapS[0];
+  g.mapS[3] = g.mapS[2];
   g.units = reinterpret_cast<const int4*>(ws + p.units2);
   g.num_units_dev = reinterpret_cast<const int*>(ws + p.nunits) + 1;
   g.roww = reinterpret_cast<const float*>(ws + p.roww);
@@ -184,6 +244,15 @@ int run_down(const Plan& p, const DeviceInfo& di, const void* Wd, const void* Ws
   g.timeout_ns = kWaitTimeoutNs;
   g.weights_evict_first = p.weights_evict_first;
   int stages = 0;
+  if (f8) {
+    int raw = 0, tok = 0;
+    g.nbuf = (2 * p.nmax2 <= 256) ? 2 : 1;
+    const size_t smem = gemm_f8_smem_bytes(kModeDown, p.nmax2, &stages, &tok, &raw);
+    g.stages = stages;
+    g.tok_stages = tok;
+    g.raw_stages = raw;
+    return launch_gemm(kModeDown, g, di.sms, smem, st, true);
+  }
   if (p.pair2) {
     g.nbuf = (p.nmax2 <= 256) ? 2 : 1;          // one accumulator per CTA
     const size_t smem = gemm_pair_smem_bytes(kModeDown, p.nmax2, &stages);
@@ -220,9 +289,8 @@ int check_expert_args(const Plan& p, const void* Wg, const void* Wu, const void*
 
 // Steps a3..a7 on a routing already in topk_idx / topk_w.
 int experts_impl(const Plan& p, const DeviceInfo& di, const void* x, const int32_t* topk_idx, const float* topk_w,
-                 const void* W_gate, const void* W_up, const void* W_down, const void* W_shared_gate,
-                 const void* W_shared_up, const void* W_shared_down, const void* W_shared_gate_vec, void* out,
-                 char* ws, cudaStream_t st) {
+                 Wt W_gate, Wt W_up, Wt W_down, Wt W_shared_gate, Wt W_shared_up, Wt W_shared_down,
+                 const void* W_shared_gate_vec, void* out, char* ws, cudaStream_t st) {
   int rc = launch_permute(p, topk_idx, topk_w, ws, st);
   if (rc == MOE_OK) rc = run_gate_up(p, di, x, W_gate, W_up, W_shared_gate, W_shared_up, ws, st);
   if (rc == MOE_OK) rc = run_down(p, di, W_down, W_shared_down, ws, st);
@@ -231,9 +299,8 @@ int experts_impl(const Plan& p, const DeviceInfo& di, const void* x, const int32
 }
 
 int forward_impl(const Plan& p, const DeviceInfo& di, const void* x, const void* W_router,
-                 const float* expert_bias, const void* W_gate, const void* W_up, const void* W_down,
-                 const void* W_shared_gate, const void* W_shared_up, const void* W_shared_down,
-                 const void* W_shared_gate_vec, int score_fn, int norm_topk, float route_scale, void* out,
+                 const float* expert_bias, Wt W_gate, Wt W_up, Wt W_down, Wt W_shared_gate, Wt W_shared_up,
+                 Wt W_shared_down, const void* W_shared_gate_vec, int score_fn, int norm_topk, float route_scale, void* out,
                  int32_t* topk_idx, float* topk_w, char* ws, cudaStream_t st) {
   int rc = run_route(p, di, x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w, ws, st);
   if (rc == MOE_OK)
@@ -241,6 +308,22 @@ int forward_impl(const Plan& p, const DeviceInfo& di, const void* x, const void*
                       W_shared_gate_vec, out, ws, st);
   return rc;
 }
+
+bool f8_given(const moe_fp8_weight* w) { return w && w->codes && w->scales; }
+bool f8_aligned(const moe_fp8_weight* w) { return aligned16(w->codes) && aligned16(w->scales); }
+
+int check_f8_expert_args(const Plan& p, const moe_fp8_weight* Wg, const moe_fp8_weight* Wu,
+                         const moe_fp8_weight* Wd, const moe_fp8_weight* Wsg, const moe_fp8_weight* Wsu,
+                         const moe_fp8_weight* Wsd) {
+  if (!f8_given(Wg) || !f8_given(Wu) || !f8_given(Wd)) return MOE_ERR_INVALID_ARG;
+  if (p.S > 0 && (!f8_given(Wsg) || !f8_given(Wsu) || !f8_given(Wsd))) return MOE_ERR_INVALID_ARG;
+  if (p.S == 0 && (Wsg || Wsu || Wsd)) return MOE_ERR_INVALID_ARG;
+  if (!f8_aligned(Wg) || !f8_aligned(Wu) || !f8_aligned(Wd)) return MOE_ERR_UNSUPPORTED;
+  if (p.S > 0 && (!f8_aligned(Wsg) || !f8_aligned(Wsu) || !f8_aligned(Wsd))) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+Wt wt(const moe_fp8_weight* w) { return w ? Wt(w->codes, w->scales) : Wt(); }
 
 int check_gate_vec(const Plan& p, const void* W_shared_gate_vec) {
   if (!W_shared_gate_vec) return MOE_OK;
@@ -538,6 +621,63 @@ int moe_forward_host(const moe_shape* shape, const void* x_host, const void* W_r
       cudaMemcpyAsync(topk_w_host, wd, tkbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+int moe_forward_fp8(const moe_shape* shape, const void* x, const void* W_router, const float* expert_bias,
+                    const moe_fp8_weight* W_gate, const moe_fp8_weight* W_up, const moe_fp8_weight* W_down,
+                    const moe_fp8_weight* W_shared_gate, const moe_fp8_weight* W_shared_up,
+                    const moe_fp8_weight* W_shared_down, const void* W_shared_gate_vec, int score_fn, int norm_topk,
+                    float route_scale, void* out, int32_t* topk_idx, float* topk_w, void* workspace,
+                    size_t workspace_bytes, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_route_args(x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w)) != MOE_OK)
+    return rc;
+  if ((rc = check_f8_expert_args(p, W_gate, W_up, W_down, W_shared_gate, W_shared_up, W_shared_down)) != MOE_OK)
+    return rc;
+  if (!out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out)) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_gate_vec(p, W_shared_gate_vec)) != MOE_OK) return rc;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return forward_impl(p, di, x, W_router, expert_bias, wt(W_gate), wt(W_up), wt(W_down), wt(W_shared_gate),
+                      wt(W_shared_up), wt(W_shared_down), W_shared_gate_vec, score_fn, norm_topk, route_scale, out,
+                      topk_idx, topk_w, static_cast<char*>(workspace), as_stream(stream));
+}
+
+int moe_expert_gate_up_fp8(const moe_shape* shape, const void* x, const moe_fp8_weight* W_gate,
+                           const moe_fp8_weight* W_up, const moe_fp8_weight* W_shared_gate,
+                           const moe_fp8_weight* W_shared_up, void* workspace, size_t workspace_bytes,
+                           moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if (!x || !f8_given(W_gate) || !f8_given(W_up)) return MOE_ERR_INVALID_ARG;
+  if (p.S > 0 && (!f8_given(W_shared_gate) || !f8_given(W_shared_up))) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !f8_aligned(W_gate) || !f8_aligned(W_up) ||
+      (p.S > 0 && (!f8_aligned(W_shared_gate) || !f8_aligned(W_shared_up))))
+    return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return run_gate_up(p, di, x, wt(W_gate), wt(W_up), p.S > 0 ? wt(W_shared_gate) : Wt(),
+                     p.S > 0 ? wt(W_shared_up) : Wt(), static_cast<char*>(workspace), as_stream(stream));
+}
+
+int moe_expert_down_fp8(const moe_shape* shape, const moe_fp8_weight* W_down, const moe_fp8_weight* W_shared_down,
+                        void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p);
+  if (rc != MOE_OK) return rc;
+  if (!f8_given(W_down) || (p.S > 0 && !f8_given(W_shared_down))) return MOE_ERR_INVALID_ARG;
+  if (!f8_aligned(W_down) || (p.S > 0 && !f8_aligned(W_shared_down))) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return run_down(p, di, wt(W_down), p.S > 0 ? wt(W_shared_down) : Wt(), static_cast<char*>(workspace),
+                  as_stream(stream));
 }
 
 int moe_rmsnorm(const moe_shape* shape, const void* x, const void* norm_gain, float eps, void* x_norm,

@@ -25,6 +25,8 @@
 // timeout in the workspace error word, drains its own copies and MMAs, frees
 // its tensor memory and returns.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "moe_internal.h"
 #include "moe_ptx.cuh"
@@ -38,16 +40,26 @@ constexpr int kGatherThreads = 32 * kGatherWarps;
 // Epilogue warps: 4 for the router (one per TMEM lane quarter), 8 for the
 // expert GEMMs (two per lane quarter, splitting the columns).
 __host__ __device__ constexpr int epi_warps_of(int mode) { return mode == kModeRouter ? 4 : 8; }
-__host__ __device__ constexpr int threads_of(int mode) {
-  return 64 + 32 * epi_warps_of(mode) + (mode == kModeGateUp ? kGatherThreads : 0);
+// Block-scaled FP8 weights: warps that widen each landed FP8 tile to bf16.
+constexpr int kConvWarps = 8;
+constexpr int kConvThreads = 32 * kConvWarps;
+// FP8 down GEMM: one warp loads the token rows (H) into the token ring.
+__host__ __device__ constexpr int threads_of(int mode, bool f8 = false) {
+  return 64 + 32 * epi_warps_of(mode) + (mode == kModeGateUp ? kGatherThreads : 0) +
+         (f8 ? kConvThreads + (mode == kModeDown ? 32 : 0) : 0);
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kATileBytes = kTileRows * 128;   // 128 weight rows x 64 bf16
 constexpr int kEpiBytes = 8192;                      // transpose staging, shared by the epilogue warps
 constexpr int kMaxStages = 8;
 constexpr int kSmemAlign = 1024;
-constexpr int kSmemTail = 512;                       // barriers, TMEM slot, abort flag
+constexpr int kSmemTail = 768;                       // barriers, TMEM slot, abort flag
 constexpr int kMaxTmemBufs = 8;                      // accumulator buffers (router: 8 x 64 columns)
+constexpr int kMaxRawStages = 12;                    // FP8: stages of the landed-tile ring
+constexpr int kMaxTokStages = 8;                     // FP8: stages of the token ring
+constexpr uint32_t kRawTileBytes = kTileRows * kTileK;           // 128 rows x 64 FP8 codes
+constexpr uint32_t kScaleTileBytes = kTileRows * (kTileK / 32);  // their scales: [2 blocks][128 rows]
+constexpr uint32_t kRawTile = kRawTileBytes + kScaleTileBytes;
 constexpr int kRouterDrainKB = 2;                    // router: k-blocks accumulated in TMEM per drain
 constexpr int kRouterMaxN = 128;                     // router: tokens per unit (fp32 sums in registers)
 
@@ -92,12 +104,101 @@ __device__ __forceinline__ float pick8(const float (&v)[8], int j) {
   return r;
 }
 
+// ---- FP8 -> bf16 widening (exact) ----
+// Integer path (the common case).  An E4M3 code s.eeee.mmm placed at bits
+// 15 / 10..7 / 6..4 of a bf16 is the bf16 e4m3(code) * 2^-120, subnormal codes
+// included (exponent field 0 is subnormal in both formats, with the same
+// mantissa scaling).  Multiplying by the bf16 2^(u-7) then gives
+// e4m3(code) * 2^(u-127) exactly whenever that is representable.  Per pair
+// of codes: one byte permute, one shift, two logic ops and one packed bf16
+// multiply, all on full-rate pipes.  2^(u-7) is a bf16 only for u <= 134;
+// larger scale bytes take the conversion-instruction path below.
+__device__ __forceinline__ uint32_t e4m3x2_placed(uint32_t y) {   // y: codes in the high bytes of its halves
+  return ((y >> 4) & 0x07F007F0u) | (y & 0x80008000u);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&a), *reinterpret_cast<const __nv_bfloat162*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// 16 codes (one 16-byte chunk, lowest address first) -> 16 bf16 in two chunks;
+// s2 = the bf16 2^(u-7) in both halves.
+__device__ __forceinline__ void fp8x16_to_bf16_int(const uint4 v, uint32_t s2, uint4& lo, uint4& hi) {
+  lo.x = bf16x2_mul(e4m3x2_placed(__byte_perm(v.x, 0u, 0x1404)), s2);
+  lo.y = bf16x2_mul(e4m3x2_placed(__byte_perm(v.x, 0u, 0x3424)), s2);
+  lo.z = bf16x2_mul(e4m3x2_placed(__byte_perm(v.y, 0u, 0x1404)), s2);
+  lo.w = bf16x2_mul(e4m3x2_placed(__byte_perm(v.y, 0u, 0x3424)), s2);
+  hi.x = bf16x2_mul(e4m3x2_placed(__byte_perm(v.z, 0u, 0x1404)), s2);
+  hi.y = bf16x2_mul(e4m3x2_placed(__byte_perm(v.z, 0u, 0x3424)), s2);
+  hi.z = bf16x2_mul(e4m3x2_placed(__byte_perm(v.w, 0u, 0x1404)), s2);
+  hi.w = bf16x2_mul(e4m3x2_placed(__byte_perm(v.w, 0u, 0x3424)), s2);
+}
+
+// Conversion-instruction path, any scale byte: an E4M3 code becomes an fp16
+// exactly (hardware conversion), an fp16 becomes an fp32 exactly, the block
+// scale 2^(u-127) multiplies exactly, and a value with at most 4 significant
+// bits rounds to bf16 exactly.
+__device__ __forceinline__ float ue8m0_scale(uint32_t u) {
+  return __uint_as_float(u == 0 ? 0x00400000u : (u == 255 ? 0x7FC00000u : u << 23));
+}
+
+__device__ __forceinline__ uint32_t fp8x2_to_bf16x2(uint32_t two, float sc) {
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+__device__ __forceinline__ void fp8x16_to_bf16_cvt(const uint4 v, float sc, uint4& lo, uint4& hi) {
+  lo.x = fp8x2_to_bf16x2(v.x & 0xFFFFu, sc);
+  lo.y = fp8x2_to_bf16x2(v.x >> 16, sc);
+  lo.z = fp8x2_to_bf16x2(v.y & 0xFFFFu, sc);
+  lo.w = fp8x2_to_bf16x2(v.y >> 16, sc);
+  hi.x = fp8x2_to_bf16x2(v.z & 0xFFFFu, sc);
+  hi.y = fp8x2_to_bf16x2(v.z >> 16, sc);
+  hi.z = fp8x2_to_bf16x2(v.w & 0xFFFFu, sc);
+  hi.w = fp8x2_to_bf16x2(v.w >> 16, sc);
+}
+
+// Widens one 32-code block - half h of row r of a landed FP8 tile, codes at
+// src (the row's 64 codes), scale byte s - into row r of the
+// 128-byte-swizzled bf16 tile at dst.  With threads (r, h) interleaved along
+// the warp, each 8-thread shared-memory wavefront covers 4 rows x 2 halves:
+// the stores hit 8 different bank groups and the loads 4 (2-way).
+__device__ __forceinline__ void widen_half(const uint8_t* src, uint32_t s, uint8_t* dst, int r, int h) {
+  const uint4 v0 = *reinterpret_cast<const uint4*>(src + 32 * h);
+  const uint4 v1 = *reinterpret_cast<const uint4*>(src + 32 * h + 16);
+  uint8_t* drow = dst + r * 128;
+  const int sw = r & 7;
+  uint4 a, b, c, d;
+  if (s <= 134u) {
+    const uint32_t e = (s + 120u) << 7;    // bf16 bits of 2^(s-7)
+    fp8x16_to_bf16_int(v0, e | (e << 16), a, b);
+    fp8x16_to_bf16_int(v1, e | (e << 16), c, d);
+  } else {
+    const float sc = ue8m0_scale(s);
+    fp8x16_to_bf16_cvt(v0, sc, a, b);
+    fp8x16_to_bf16_cvt(v1, sc, c, d);
+  }
+  *reinterpret_cast<uint4*>(drow + (((4 * h + 0) ^ sw) << 4)) = a;
+  *reinterpret_cast<uint4*>(drow + (((4 * h + 1) ^ sw) << 4)) = b;
+  *reinterpret_cast<uint4*>(drow + (((4 * h + 2) ^ sw) << 4)) = c;
+  *reinterpret_cast<uint4*>(drow + (((4 * h + 3) ^ sw) << 4)) = d;
+}
+
 // SiLU(z) = z * sigmoid(z) with the fast exponential and division; the
 // exponent is clamped so the denominator stays finite (|result| < 1e-32 there).
 __device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(fminf(-z, 80.0f))); }
 
-template <int MODE>
-__global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __grid_constant__ GemmParams p) {
+// F8: the routed and shared expert weights are block-scaled FP8 (codes plus
+// one power-of-two scale per 32 codes along K).  The producer lands code and
+// scale tiles in a ring of their own; kConvWarps converter warps widen each
+// tile to bf16 into the MMA stage (exact), so the tensor cores and the rest
+// of the kernel are those of the bf16 path while HBM moves half the bytes.
+template <int MODE, bool F8>
+__global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const __grid_constant__ GemmParams p) {
+  static_assert(!F8 || MODE != kModeRouter, "the router weights stay bf16");
   // A tiles (and accumulators) per unit: gate/up: the gate and the up tile of
   // the same 128 rows; down: two consecutive 128-row blocks of W_down (a
   // 256-row unit, so each token row loaded serves 256 outputs); router: one.
@@ -108,24 +209,53 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
       (reinterpret_cast<uintptr_t>(smem_raw) + (kSmemAlign - 1)) & ~static_cast<uintptr_t>(kSmemAlign - 1));
   const int nmax = p.nmax;
   const int S = p.stages;
-  const uint32_t stage_bytes = NA * kATileBytes + static_cast<uint32_t>(nmax) * 128u;
-  uint8_t* epi = smem + static_cast<size_t>(S) * stage_bytes;
+  const uint32_t tok_bytes = static_cast<uint32_t>(nmax) * 128u;
+  // bf16: each MMA stage holds the weight tiles and the token tile.  FP8:
+  // three rings - MMA stages of widened weight tiles (S), token tiles (TS),
+  // and the landing ring of code + scale tiles (R) - so that token loads run
+  // as far ahead as the bf16 path's, however few widened stages fit.
+  const uint32_t stage_bytes = NA * kATileBytes + (F8 ? 0u : tok_bytes);
+  const int TS = F8 ? p.tok_stages : 0;
+  const int R = F8 ? p.raw_stages : 0;
+  constexpr uint32_t raw_stage_bytes = NA * kRawTile;
+  uint8_t* tokring = smem + static_cast<size_t>(S) * stage_bytes;
+  uint8_t* raw = tokring + static_cast<size_t>(TS) * tok_bytes;
+  uint8_t* epi = raw + static_cast<size_t>(R) * raw_stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(epi + kEpiBytes);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + kMaxTmemBufs;
   uint64_t* drain = tempty + kMaxTmemBufs;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* raw_full = drain + 1;
+  uint64_t* raw_empty = raw_full + R;
+  uint64_t* tok_full = raw_empty + R;
+  uint64_t* tok_empty = tok_full + TS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tok_empty + TS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // FP8 warps after the epilogue (and gather) warps: down: one token loader,
+  // then the converters; gate/up: the converters.
+  constexpr int kTokWarp = 2 + epi_warps_of(MODE);
+  constexpr int kConvBase =
+      2 + epi_warps_of(MODE) + (MODE == kModeGateUp ? kGatherWarps : 0) + (F8 && MODE == kModeDown ? 1 : 0);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      // gate/up: the weight-tile producer's arrival plus one per gathering thread
-      mbar_init(full + s, MODE == kModeGateUp ? 1 + kGatherThreads : 1);
+      // bf16: the producer's arrival plus (gate/up) one per gathering thread;
+      // FP8: one per converter warp
+      mbar_init(full + s, F8 ? kConvWarps : 1 + (MODE == kModeGateUp ? kGatherThreads : 0));
       mbar_init(empty + s, 1);
+    }
+    for (int r = 0; r < R; ++r) {
+      mbar_init(raw_full + r, 1);
+      mbar_init(raw_empty + r, kConvWarps);
+    }
+    for (int t = 0; t < TS; ++t) {
+      // gate/up: one per gathering thread; down: the token loader's arrival
+      mbar_init(tok_full + t, MODE == kModeGateUp ? kGatherThreads : 1);
+      mbar_init(tok_empty + t, 1);
     }
     for (int b = 0; b < kMaxTmemBufs; ++b) {
       mbar_init(tfull + b, 1);
@@ -137,6 +267,8 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
   }
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < 2 * NA; ++i) prefetch_tensormap(&p.mapA[i]);
+    if (F8)
+      for (int i = 0; i < 2 * NA; ++i) prefetch_tensormap(&p.mapS[i]);
     if (MODE != kModeGateUp)
       for (int i = 0; i < 4; ++i) prefetch_tensormap(&p.mapB[0][i]);
   }
@@ -159,6 +291,10 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
     const uint64_t pol_a = (MODE == kModeRouter || !p.weights_evict_first) ? policy_evict_last()
                                                                            : policy_evict_first();
     const uint64_t pol_b = policy_evict_last();
+    // the ring this warp fills: the MMA stages, or (FP8) the landing ring
+    uint64_t* pfull = F8 ? raw_full : full;
+    uint64_t* pempty = F8 ? raw_empty : empty;
+    const int PS = F8 ? R : S;
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued = 0;
@@ -180,21 +316,38 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
       int got = 1;
       if (lane == 0) {
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
+          if (!mbar_wait(&pempty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
             got = 0;
             break;
           }
-          const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
-          const uint32_t fb = smem_u32(&full[stage]);
-          mbar_arrive_expect_tx(&full[stage], tx_bytes);
+          if constexpr (F8) {
+            // code tile(s) and their scales into the landing ring; the
+            // converter warps widen them into the MMA stage
+            const uint32_t rbase = smem_u32(raw + static_cast<size_t>(stage) * raw_stage_bytes);
+            const uint32_t fb = smem_u32(&raw_full[stage]);
+            const CUtensorMap* mS = &p.mapS[sh ? 2 : 0];
+            mbar_arrive_expect_tx(&raw_full[stage], raw_stage_bytes);
 #pragma unroll
-          for (int a = 0; a < NA; ++a)
-            tma_load_3d_hint(sbase + a * kATileBytes, (MODE == kModeDown) ? mA : mA + a, fb, kb * kTileK,
-                             un.wb * kWbRows + ((MODE == kModeDown) ? a * kTileRows : 0), a_c2, pol_a);
-          if (MODE != kModeGateUp)
-            tma_load_rows<false>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, un.n, pol_b);
+            for (int a = 0; a < NA; ++a) {
+              const int wrow = un.wb * kWbRows + ((MODE == kModeDown) ? a * kTileRows : 0);
+              tma_load_3d_hint(rbase + a * kRawTile, (MODE == kModeDown) ? mA : mA + a, fb, kb * kTileK, wrow,
+                               a_c2, pol_a);
+              tma_load_3d(rbase + a * kRawTile + kRawTileBytes, (MODE == kModeDown) ? mS : mS + a, fb, wrow,
+                          kb * (kTileK / 32), a_c2);
+            }
+          } else {
+            const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+            const uint32_t fb = smem_u32(&full[stage]);
+            mbar_arrive_expect_tx(&full[stage], tx_bytes);
+#pragma unroll
+            for (int a = 0; a < NA; ++a)
+              tma_load_3d_hint(sbase + a * kATileBytes, (MODE == kModeDown) ? mA : mA + a, fb, kb * kTileK,
+                               un.wb * kWbRows + ((MODE == kModeDown) ? a * kTileRows : 0), a_c2, pol_a);
+            if (MODE != kModeGateUp)
+              tma_load_rows<false>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, un.n, pol_b);
+          }
           ++issued;
-          if (++stage == S) {
+          if (++stage == PS) {
             stage = 0;
             phase ^= 1u;
           }
@@ -203,12 +356,12 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) ok = false;
     }
-    // Leave no copy in flight: the last min(S, issued) stages armed.
+    // Leave no copy in flight: the last min(PS, issued) stages armed.
     if (lane == 0) {
-      const uint32_t outstanding = issued < static_cast<uint32_t>(S) ? issued : static_cast<uint32_t>(S);
+      const uint32_t outstanding = issued < static_cast<uint32_t>(PS) ? issued : static_cast<uint32_t>(PS);
       for (uint32_t i = 1; i <= outstanding; ++i) {
         const uint32_t I = issued - i;
-        mbar_wait_drain(&full[I % S], (I / S) & 1u, p.timeout_ns);
+        mbar_wait_drain(&pfull[I % PS], (I / PS) & 1u, p.timeout_ns);
       }
     }
   } else if (warp == 1) {
@@ -216,6 +369,8 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      int tstage = 0;                 // FP8: token ring
+      uint32_t tphase = 0;
       uint32_t ucount = 0;
       bool any = false;
       bool ok = true;
@@ -277,16 +432,19 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
           const uint32_t idesc = idesc_bf16_f32(kTileRows, un.n);
           const uint32_t dcol = tmem_base + static_cast<uint32_t>(buf * NA * nmax);
           for (int kb = 0; kb < KB; ++kb) {
-            if (!mbar_wait(&full[stage], phase, abort_flag, p.err, p.timeout_ns)) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, p.err, p.timeout_ns) ||
+                (F8 && !mbar_wait(&tok_full[tstage], tphase, abort_flag, p.err, p.timeout_ns))) {
               ok = false;
               break;
             }
             tc_fence_after();
-            // Token rows written by cp.async (generic proxy) are read by the
-            // tensor cores (async proxy).
-            if (MODE == kModeGateUp) fence_proxy_async_smem();
+            // Token rows written by cp.async and (FP8) weight tiles written by
+            // the converters (generic proxy) are read by the tensor cores
+            // (async proxy).
+            if (MODE == kModeGateUp || F8) fence_proxy_async_smem();
             const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
-            const uint64_t bdesc = sw128_kmajor_desc(sbase + NA * kATileBytes);
+            const uint64_t bdesc = sw128_kmajor_desc(
+                F8 ? smem_u32(tokring + static_cast<size_t>(tstage) * tok_bytes) : sbase + NA * kATileBytes);
             uint64_t adesc[NA];
 #pragma unroll
             for (int a = 0; a < NA; ++a) adesc[a] = sw128_kmajor_desc(sbase + a * kATileBytes);
@@ -303,6 +461,13 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
               stage = 0;
               phase ^= 1u;
             }
+            if (F8) {
+              tc_commit(&tok_empty[tstage]);
+              if (++tstage == TS) {
+                tstage = 0;
+                tphase ^= 1u;
+              }
+            }
           }
           if (!ok) break;
           tc_commit(&tfull[buf]);
@@ -316,7 +481,96 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
       }
     }
     __syncwarp();
-  } else if (MODE == kModeGateUp && warp >= 2 + epi_warps_of(MODE)) {
+  } else if (F8 && warp >= kConvBase) {
+    // ------------------------------------------------------------ FP8 -> bf16
+    // Thread c widens block (c & 1) of row (c >> 1) of every landed code
+    // tile into the MMA stage.
+    const int c = threadIdx.x - 32 * kConvBase;
+    const int crow = c >> 1, chalf = c & 1;
+    int rs = 0, ms = 0;              // landing-ring and MMA-ring positions
+    uint32_t rph = 0, mph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      const Unit un = get_unit<MODE>(p, u);
+      const bool sh = un.g >= p.E;
+      const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
+      const int KB = K / kTileK;
+      for (int kb = 0; kb < KB; ++kb) {
+        int got = 1;
+        if (lane == 0)
+          got = (mbar_wait(&raw_full[rs], rph, abort_flag, p.err, p.timeout_ns) &&
+                 mbar_wait(&empty[ms], mph ^ 1u, abort_flag, p.err, p.timeout_ns))
+                    ? 1
+                    : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          ok = false;
+          break;
+        }
+        uint8_t* sb = smem + static_cast<size_t>(ms) * stage_bytes;
+        const uint8_t* rt = raw + static_cast<size_t>(rs) * raw_stage_bytes;
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+          const uint8_t* q = rt + a * kRawTile;
+          widen_half(q + crow * kTileK, q[kRawTileBytes + chalf * kTileRows + crow], sb + a * kATileBytes, crow,
+                     chalf);
+        }
+        fence_proxy_async_smem();      // generic-proxy stores -> tensor-core reads
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&raw_empty[rs]);
+          mbar_arrive(&full[ms]);
+        }
+        if (++rs == R) {
+          rs = 0;
+          rph ^= 1u;
+        }
+        if (++ms == S) {
+          ms = 0;
+          mph ^= 1u;
+        }
+      }
+    }
+  } else if (F8 && MODE == kModeDown && warp == kTokWarp) {
+    // ------------------------------------------------------------ FP8 down: token rows
+    // H rows of each k-block into the token ring, up to TS k-blocks ahead.
+    if constexpr (F8) if (lane == 0) {
+      const uint64_t pol_b = policy_evict_last();
+      int ts = 0;
+      uint32_t tph = 0, issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const Unit un = get_unit<MODE>(p, u);
+        const bool sh = un.g >= p.E;
+        const int sidx = sh ? un.g - p.E : 0;
+        const int KB = (sh ? p.fs : p.f) / kTileK;
+        const CUtensorMap* mB = p.mapB[sh ? 1 : 0];
+        const int brow0 = sh ? sidx * p.Tp + un.row0 : un.row0;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&tok_empty[ts], tph ^ 1u, abort_flag, p.err, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&tok_full[ts], static_cast<uint32_t>(un.n) * 128u);
+          tma_load_rows<false>(smem_u32(tokring + static_cast<size_t>(ts) * tok_bytes), mB, smem_u32(&tok_full[ts]),
+                               kb * kTileK, brow0, un.n, pol_b);
+          ++issued;
+          if (++ts == TS) {
+            ts = 0;
+            tph ^= 1u;
+          }
+        }
+      }
+      // leave no copy in flight
+      const uint32_t outstanding = issued < static_cast<uint32_t>(TS) ? issued : static_cast<uint32_t>(TS);
+      for (uint32_t i = 1; i <= outstanding; ++i) {
+        const uint32_t I = issued - i;
+        mbar_wait_drain(&tok_full[I % TS], (I / TS) & 1u, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (MODE == kModeGateUp && warp >= 2 + epi_warps_of(MODE) &&
+             warp < 2 + epi_warps_of(MODE) + kGatherWarps) {
     // ------------------------------------------------------------ row gather
     // Thread g copies 16-byte chunk (g & 7) of rows (g >> 3) + 16 i of the
     // token tile, i < n / 16, into the 128-byte-swizzled slot: chunk c of row
@@ -325,6 +579,10 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
     const int part = g & 7;
     const int r0 = g >> 3;
     const uint64_t pol_x = policy_evict_last();     // x rows are gathered by every weight block
+    // the ring the token tiles go to: the MMA stages, or (FP8) the token ring
+    uint64_t* gfull = F8 ? tok_full : full;
+    uint64_t* gempty = F8 ? tok_empty : empty;
+    const int GS = F8 ? TS : S;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -342,13 +600,14 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
       const int KB = p.d / kTileK;
       for (int kb = 0; kb < KB; ++kb) {
         int got = 1;
-        if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+        if (lane == 0) got = mbar_wait(&gempty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) {
           ok = false;
           break;
         }
-        const uint32_t bbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + NA * kATileBytes;
+        const uint32_t bbase = F8 ? smem_u32(tokring + static_cast<size_t>(stage) * tok_bytes)
+                                  : smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + NA * kATileBytes;
         const __nv_bfloat16* src0 = reinterpret_cast<const __nv_bfloat16*>(p.x) + kb * kTileK + part * 8;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -358,8 +617,8 @@ __global__ void __launch_bounds__(threads_of(MODE), 1) moe_gemm_kernel(const __g
                         pol_x);
           }
         }
-        cp_async_mbar_arrive_noinc(&full[stage]);
-        if (++stage == S) {
+        cp_async_mbar_arrive_noinc(&gfull[stage]);
+        if (++stage == GS) {
           stage = 0;
           phase ^= 1u;
         }
@@ -971,29 +1230,60 @@ int launch_gemm_pair(int mode, const GemmParams& prm, int grid, size_t smem, cud
   }
 }
 
-template <int MODE>
+size_t gemm_f8_smem_bytes(int mode, int nmax, int* stages, int* tok_stages, int* raw_stages) {
+  const int NA = 2;   // gate/up and down both stage two weight tiles
+  const size_t stage_bytes = NA * static_cast<size_t>(kATileBytes);
+  const size_t tok_bytes = static_cast<size_t>(nmax) * 128;
+  const size_t raw_stage = NA * static_cast<size_t>(kRawTile);
+  const size_t fixed = kSmemAlign + kEpiBytes + kSmemTail;
+  const size_t budget = 232448;
+  (void)mode;
+  const int s = 2;    // the converters fill one MMA stage while the tensor cores read the other
+  int ts = static_cast<int>(65536 / tok_bytes);   // 64 KB of token tiles
+  if (ts < 2) ts = 2;
+  if (ts > kMaxTokStages) ts = kMaxTokStages;
+  int r = static_cast<int>((budget - fixed - s * stage_bytes - ts * tok_bytes) / raw_stage);
+  if (r > kMaxRawStages) r = kMaxRawStages;
+  if (stages) *stages = s;
+  if (tok_stages) *tok_stages = ts;
+  if (raw_stages) *raw_stages = r;
+  return fixed + s * stage_bytes + ts * tok_bytes + static_cast<size_t>(r) * raw_stage;
+}
+
+template <int MODE, bool F8>
 static int launch_mode(const GemmParams& prm, int grid, size_t smem, cudaStream_t st) {
   static int configured[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
   if (configured[dev] < static_cast<int>(smem)) {
-    if (cudaFuncSetAttribute(moe_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(moe_gemm_kernel<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return MOE_ERR_CUDA;
     configured[dev] = static_cast<int>(smem);
   }
-  return launch_chained(moe_gemm_kernel<MODE>, dim3(grid), dim3(threads_of(MODE)), smem, st, prm) == cudaSuccess
+  return launch_chained(moe_gemm_kernel<MODE, F8>, dim3(grid), dim3(threads_of(MODE, F8)), smem, st, prm) ==
+                 cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
 
-int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st) {
+int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st, bool f8) {
   if (grid < 1) return MOE_OK;
+  if (f8) {
+    if (prm.raw_stages < 2 || prm.raw_stages > kMaxRawStages || prm.stages != 2 || prm.tok_stages < 2 ||
+        prm.tok_stages > kMaxTokStages)
+      return MOE_ERR_INVALID_ARG;
+    switch (mode) {
+      case kModeGateUp: return launch_mode<kModeGateUp, true>(prm, grid, smem, st);
+      case kModeDown: return launch_mode<kModeDown, true>(prm, grid, smem, st);
+      default: return MOE_ERR_INVALID_ARG;
+    }
+  }
   switch (mode) {
-    case kModeRouter: return launch_mode<kModeRouter>(prm, grid, smem, st);
-    case kModeGateUp: return launch_mode<kModeGateUp>(prm, grid, smem, st);
-    case kModeDown: return launch_mode<kModeDown>(prm, grid, smem, st);
+    case kModeRouter: return launch_mode<kModeRouter, false>(prm, grid, smem, st);
+    case kModeGateUp: return launch_mode<kModeGateUp, false>(prm, grid, smem, st);
+    case kModeDown: return launch_mode<kModeDown, false>(prm, grid, smem, st);
     default: return MOE_ERR_INVALID_ARG;
   }
 }

@@ -108,10 +108,17 @@ struct GemmParams {
   int nmax, stages, nbuf, router_nwb;
   uint64_t timeout_ns;
   int weights_evict_first;  // 1: each weight tile is read by one unit (experts fit one token run)
+  // block-scaled FP8 expert weights: mapA are then the code tensors (uint8,
+  // tiles of 128 rows x 64 codes) and mapS their scales ([G, K/32, rows] uint8,
+  // tiles of 128 rows x 2 blocks); raw_stages = depth of the landing ring
+  CUtensorMap mapS[4];
+  int raw_stages, tok_stages;
 };
 
-int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st);
+int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st, bool f8 = false);
 size_t gemm_smem_bytes(int mode, int nmax, int* stages);
+// FP8 expert GEMMs: MMA stages and landing-ring stages for an nmax
+size_t gemm_f8_smem_bytes(int mode, int nmax, int* stages, int* tok_stages, int* raw_stages);
 // CTA-pair (cta_group::2) expert GEMMs; grid is rounded down to an even count.
 int launch_gemm_pair(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st);
 size_t gemm_pair_smem_bytes(int mode, int nmax, int* stages);

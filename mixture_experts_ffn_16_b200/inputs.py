@@ -47,6 +47,7 @@ class MoEConfig:
     skew: str = ""                     # "" | "zipf_rank"
     shared_gate: bool = False          # per-token sigmoid gate on the shared experts (Qwen3.5)
     prenorm: bool = False              # pre-norm RMSNorm (zero-centred gains) in front of the block
+    fp8: bool = False                  # expert weights also as block-scaled FP8 (quantised from the bf16 draw)
     norm_eps: float = 1e-6
     seed: int = 0
     x_std: float = 1.0
@@ -116,6 +117,11 @@ def make_inputs(cfg: MoEConfig, device="cpu", seed=None):
     W_shared_gate_vec = None
     if cfg.shared_gate and S > 0:
         W_shared_gate_vec = _randn_bf16((S, d), cfg.w_std, gen, device)
+    fp8 = {}
+    if cfg.fp8:
+        for name, w in (("W_gate", W_gate), ("W_up", W_up), ("W_down", W_down), ("W_shared_gate", W_shared_gate),
+                        ("W_shared_up", W_shared_up), ("W_shared_down", W_shared_down)):
+            fp8[name + "_f8"] = quantize_mxfp8(w) if w is not None else None
     norm_gain = None
     if cfg.prenorm:
         norm_gain = _randn_bf16((d,), 0.1, gen, device)
@@ -127,7 +133,36 @@ def make_inputs(cfg: MoEConfig, device="cpu", seed=None):
         W_router[:, 0] = offset.to(torch.bfloat16)
     return dict(x=x, W_router=W_router, expert_bias=bias, W_gate=W_gate, W_up=W_up, W_down=W_down,
                 W_shared_gate=W_shared_gate, W_shared_up=W_shared_up, W_shared_down=W_shared_down,
-                W_shared_gate_vec=W_shared_gate_vec, norm_gain=norm_gain, ranks=ranks)
+                W_shared_gate_vec=W_shared_gate_vec, norm_gain=norm_gain, ranks=ranks, **fp8)
+
+
+def quantize_mxfp8(w, block=32):
+    """bf16 weights [G, rows, K] -> (codes uint8 [G, rows, K], scales uint8 [G, K/32, rows]).
+
+    Synthetic FP8 weights: per 32-element block along K the scale is the
+    smallest power of two 2^(u-127) with max|w| / 2^(u-127) <= 448 (the largest
+    E4M3 magnitude), and each code is w / 2^(u-127) rounded to the nearest
+    E4M3 value (ties to even).  An all-zero block gets u = 127."""
+    G, rows, K = w.shape
+    if K % block:
+        raise ValueError("K must be a multiple of the block size")
+    nb = K // block
+    codes = torch.empty((G, rows, K), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((G, nb, rows), dtype=torch.uint8, device=w.device)
+    per = max(1, (1 << 26) // max(1, rows * K))
+    for g0 in range(0, G, per):
+        g1 = min(G, g0 + per)
+        wf = w[g0:g1].float().view(g1 - g0, rows, nb, block)
+        amax = wf.abs().amax(-1)                                      # [g, rows, nb]
+        m, e = torch.frexp(amax / 448.0)                              # amax/448 = m 2^e, 0.5 <= m < 1
+        ce = torch.where(m == 0.5, e - 1, e)                          # ceil(log2(amax / 448))
+        u = torch.where(amax > 0, ce + 127, torch.full_like(ce, 127)).clamp(1, 254)
+        scaled = wf / torch.exp2((u - 127).float()).unsqueeze(-1)
+        q = scaled.to(torch.float8_e4m3fn).view(torch.uint8)
+        codes[g0:g1] = q.view(g1 - g0, rows, K)
+        scales[g0:g1] = u.to(torch.uint8).permute(0, 2, 1)
+        del wf, amax, m, e, ce, u, scaled, q
+    return codes, scales
 
 
 def bf16_bits(t):

@@ -5,7 +5,8 @@ Counts only what the method must do, not what an implementation moves:
          shared rows, each 2 x f x d), down (same rows, d x f).
   bytes  every weight matrix a kernel needs read once (routed experts only if
          some token picked them), activations read once and results written
-         once, in their stored dtype.
+         once, in their stored dtype (block-scaled FP8 expert weights: one
+         byte per code plus one scale byte per 32 codes).
 """
 from __future__ import annotations
 
@@ -31,12 +32,18 @@ def measured_peaks():
         return dict(FALLBACK_PEAKS, source="fallback")
 
 
+def weight_bytes(cfg):
+    """Bytes per expert-weight element: bf16, or FP8 code + 1/32 scale byte."""
+    return 1.0 + 1.0 / 32.0 if getattr(cfg, "fp8", False) else 2.0
+
+
 def kernel_costs(cfg, touched=None):
     """Per-step algorithmic (flops, bytes) of each step of the block.
 
     touched: number of routed experts with at least one token (default: all E).
     """
     T, d, E, k, f, S, fs = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.S, cfg.fs
+    wb = weight_bytes(cfg)
     ne = E if touched is None else int(touched)
     R = T * k
     c = {}
@@ -46,10 +53,10 @@ def kernel_costs(cfg, touched=None):
     c["permute"] = (0.0, 8.0 * R * 2 + 12.0 * R)
     # a4 + a6 gate/up: weights of touched experts and shared, x, H out
     c["gate_up"] = (2.0 * (R * 2 * f * d + S * T * 2 * fs * d),
-                    2.0 * (ne * 2 * f * d + S * 2 * fs * d + T * d + R * f + S * T * fs))
+                    wb * (ne * 2 * f * d + S * 2 * fs * d) + 2.0 * (T * d + R * f + S * T * fs))
     # a5 + a6 down: W_down, H in, Y out
     c["down"] = (2.0 * (R * d * f + S * T * d * fs),
-                 2.0 * (ne * d * f + S * d * fs + R * f + S * T * fs + R * d + S * T * d))
+                 wb * (ne * d * f + S * d * fs) + 2.0 * (R * f + S * T * fs + R * d + S * T * d))
     # a7 combine: Y rows in, out written
     c["combine"] = (float((R + S * T) * d), 2.0 * ((R + S * T) * d + T * d) + 4.0 * R)
     return c
@@ -61,7 +68,8 @@ def block_cost(cfg, touched=None):
     T, d, E, k, f, S, fs = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.S, cfg.fs
     ne = E if touched is None else int(touched)
     flops = 2.0 * T * E * d + 2.0 * T * k * 3 * f * d + 2.0 * T * S * 3 * fs * d
-    bytes_ = 2.0 * (ne * 3 * f * d + S * 3 * fs * d + E * d + 2 * T * d) + 8.0 * T * k
+    bytes_ = (weight_bytes(cfg) * (ne * 3 * f * d + S * 3 * fs * d) + 2.0 * (E * d + 2 * T * d)
+              + 8.0 * T * k)
     return flops, bytes_
 
 

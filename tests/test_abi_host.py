@@ -180,3 +180,31 @@ def test_x_stage_region(lib):
     s = api.make_shape(16, 128, 8, 2, 128, 1, 128)
     off, nb = api.moe_workspace_region(s, "x_stage")
     assert nb == 16 * 128 * 2 and off % 256 == 0 and off + nb <= api.moe_workspace_bytes(s)
+
+
+def test_fp8_argument_checks(lib):
+    """FP8 entry points refuse null or half-given weights and misalignment before any device work."""
+    s = api.make_shape(16, 128, 8, 2, 128, 1, 128)
+    n = api.moe_workspace_bytes(s)
+    P = ctypes.c_void_p
+    W = api.MoeFp8Weight
+    good = W(P(4096), P(8192))
+
+    def fwd(ws6=None, shape=s, nb=n):
+        ws6 = ws6 if ws6 is not None else [good] * 6
+        ptrs = [None if w is None else ctypes.pointer(w) for w in ws6]
+        return lib.moe_forward_fp8(ctypes.byref(shape), P(4096), P(4096), None, *ptrs, None, 0, 1, 1.0,
+                                   P(4096), P(4096), P(4096), P(4096), nb, None)
+
+    assert fwd([None] + [good] * 5) == api.MOE_ERR_INVALID_ARG
+    assert fwd([W(P(4096), None)] + [good] * 5) == api.MOE_ERR_INVALID_ARG      # codes without scales
+    assert fwd([good] * 3 + [None] * 3) == api.MOE_ERR_INVALID_ARG              # S = 1 needs shared weights
+    assert fwd([W(P(4100), P(8192))] + [good] * 5) == api.MOE_ERR_UNSUPPORTED
+    assert fwd([good] * 2 + [W(P(4096), P(8200))] + [good] * 3) == api.MOE_ERR_UNSUPPORTED
+    s0 = api.make_shape(16, 128, 8, 2, 128, 0, 0)
+    assert fwd([good] * 6, shape=s0, nb=api.moe_workspace_bytes(s0)) == api.MOE_ERR_INVALID_ARG
+    assert fwd(nb=n - 1) == api.MOE_ERR_WORKSPACE
+    pg = ctypes.pointer(good)
+    assert lib.moe_expert_gate_up_fp8(ctypes.byref(s), P(4096), pg, None, pg, pg, P(4096), n, None) == \
+        api.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_down_fp8(ctypes.byref(s), pg, None, P(4096), n, None) == api.MOE_ERR_INVALID_ARG

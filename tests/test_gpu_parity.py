@@ -243,3 +243,96 @@ def test_prenorm_full_size_sampled(oracle_mod):
     host["x"] = ref_xn
     rep = check_parity(oracle_mod, cfg, host, out[tokens], idx[tokens], w[tokens], tokens=tokens)
     print(cfg.name, rep)
+
+
+# ---------------------------------------------------------------- block-scaled FP8 expert weights
+
+def _fp8_host_args(oracle_mod, inp):
+    """Oracle inputs with every expert weight replaced by the oracle's own
+    (exact) dequantisation of the FP8 codes and scales the GPU reads."""
+    host = oracle_args(inp)
+    for name in ("W_gate", "W_up", "W_down", "W_shared_gate", "W_shared_up", "W_shared_down"):
+        f8 = inp.get(name + "_f8")
+        if f8 is not None:
+            host[name] = oracle_mod.dequant_mxfp8(f8[0].cpu().numpy(), f8[1].cpu().numpy())
+    return host
+
+
+FP8 = [
+    MoEConfig("fp8_softmax_ragged", T=300, d=512, E=40, k=6, f=192, S=1, fs=320, fp8=True, seed=41),
+    MoEConfig("fp8_sigmoid_two_shared", T=257, d=384, E=24, k=4, f=256, S=2, fs=128, score_fn="sigmoid",
+              bias_std=0.1, route_scale=2.5, fp8=True, seed=42),
+    MoEConfig("fp8_decode_like", T=64, d=1024, E=64, k=10, f=512, S=1, fs=512, score_fn="sqrt_softplus",
+              bias_std=0.1, fp8=True, seed=43),
+    MoEConfig("fp8_many_rows_gated", T=2000, d=256, E=4, k=2, f=128, S=1, fs=128, shared_gate=True, fp8=True,
+              seed=44),
+    MoEConfig("fp8_no_shared_min_width", T=17, d=64, E=5, k=2, f=64, S=0, fs=0, fp8=True, seed=45),
+]
+
+
+@pytest.mark.parametrize("cfg", FP8, ids=lambda c: c.name)
+def test_fp8_weights_every_token(oracle_mod, cfg):
+    """moe_forward_fp8 against the oracle's block on the oracle's dequantised
+    weights: the widening to bf16 is exact, so the same bar as the bf16 path."""
+    _need_gpu()
+    inp = make_inputs(cfg, device="cuda")
+    out, idx, w, _ = run_gpu(cfg, inp)
+    rep = check_parity(oracle_mod, cfg, _fp8_host_args(oracle_mod, inp), out, idx, w)
+    print(cfg.name, rep)
+
+
+def test_fp8_full_size_sampled(oracle_mod):
+    cfg = MoEConfig("prefill_softmax_fp8", T=4096, d=2048, E=256, k=8, f=512, S=1, fs=512, fp8=True, seed=46)
+    _need_gpu()
+    inp = make_inputs(cfg, device="cuda")
+    out, idx, w, _ = run_gpu(cfg, inp)
+    tokens = _sample(cfg.T, 128, seed=47)
+    rep = check_parity(oracle_mod, cfg, _fp8_host_args(oracle_mod, inp), out[tokens], idx[tokens], w[tokens],
+                       tokens=tokens)
+    print(cfg.name, rep)
+
+
+def test_fp8_steps_equal_forward(oracle_mod):
+    """The FP8 step entry points, called one by one, give the forward's bits."""
+    _need_gpu()
+    cfg = FP8[0]
+    inp = make_inputs(cfg, device="cuda")
+    layer = api.MoELayer(cfg, inp)
+    out1 = layer()[0].clone()
+    out2 = layer.steps()[0].clone()
+    assert api.moe_device_status(layer.workspace) == api.MOE_OK
+    assert torch.equal(out1, out2)
+
+
+def _crafted_f8(shape_g_rows_k, codes_pool, u_pool, gen):
+    G, rows, K = shape_g_rows_k
+    pool = torch.tensor(codes_pool, dtype=torch.uint8)
+    upool = torch.tensor(u_pool, dtype=torch.uint8)
+    codes = pool[torch.randint(len(codes_pool), (G, rows, K), generator=gen)]
+    scales = upool[torch.randint(len(u_pool), (G, K // 32, rows), generator=gen)]
+    return codes.cuda(), scales.cuda()
+
+
+@pytest.mark.parametrize("kind", ["subnormal_codes", "large_scales"])
+def test_fp8_widening_edge_codes(oracle_mod, kind):
+    """Weights made only of subnormal E4M3 codes (exponent field 0, both signs),
+    or of normal codes under scale bytes above 134 (the conversion-instruction
+    path): the widened bf16 must equal the oracle's exact dequantisation, so a
+    flushed subnormal or a mis-scaled block fails."""
+    _need_gpu()
+    cfg = MoEConfig("fp8_" + kind, T=200, d=256, E=6, k=2, f=128, S=1, fs=128, fp8=True, seed=48)
+    inp = make_inputs(cfg, device="cuda")
+    g = torch.Generator().manual_seed(49)
+    if kind == "subnormal_codes":
+        codes = [c for c in range(1, 8)] + [0x80 | c for c in range(1, 8)] + [0x00, 0x80]
+        us = [129, 130, 131, 134]
+    else:
+        codes = [0x20, 0x21, 0x27, 0xA3, 0x30, 0xB5]          # 2^-3 .. 2^-1 magnitudes
+        us = [135, 136, 138, 134, 120]
+    for name, gdim, rows, K in (("W_gate", cfg.E, cfg.f, cfg.d), ("W_up", cfg.E, cfg.f, cfg.d),
+                                ("W_down", cfg.E, cfg.d, cfg.f), ("W_shared_gate", cfg.S, cfg.fs, cfg.d),
+                                ("W_shared_up", cfg.S, cfg.fs, cfg.d), ("W_shared_down", cfg.S, cfg.d, cfg.fs)):
+        inp[name + "_f8"] = _crafted_f8((gdim, rows, K), codes, us, g)
+    out, idx, w, _ = run_gpu(cfg, inp)
+    rep = check_parity(oracle_mod, cfg, _fp8_host_args(oracle_mod, inp), out, idx, w)
+    print(cfg.name, rep)
