@@ -254,8 +254,9 @@ def run_ours(args, cfg):
                           layer.topk_idx, layer.topk_w, layer.workspace, stream)
         if ev is not None:
             ev[1].record(stream)
-        api.moe_permute(s, ext_idx if external else layer.topk_idx, ext_w if external else layer.topk_w,
-                        layer.workspace, stream)
+        (api.moe_permute_fp8 if c.fp8 else api.moe_permute)(
+            s, ext_idx if external else layer.topk_idx, ext_w if external else layer.topk_w, layer.workspace,
+            stream)
         if ev is not None:
             ev[2].record(stream)
         if c.fp8:

@@ -198,8 +198,15 @@ MOE_API int moe_forward_fp8(const moe_shape *shape,
                 void *out, int32_t *topk_idx, float *topk_w,
                 void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
-/* The FP8 forms of the two expert steps (a4 + a6, a5 + a6), for callers that
- * run the steps one by one. */
+/* The FP8 forms of the permute and the two expert steps (a3, a4 + a6, a5 + a6),
+ * for callers that run the steps one by one: moe_route, moe_permute_fp8,
+ * moe_expert_gate_up_fp8, moe_expert_down_fp8, moe_combine.  The FP8 GEMMs
+ * take token runs of at most 128 rows and no CTA pairs, so their work lists
+ * differ from the bf16 ones; an expert step that meets lists built for the
+ * other format does nothing and moe_device_status reports
+ * MOE_ERR_INVALID_ARG. */
+MOE_API int moe_permute_fp8(const moe_shape *shape, const int32_t *topk_idx, const float *topk_w,
+                void *workspace, size_t workspace_bytes, moe_stream_t stream);
 MOE_API int moe_expert_gate_up_fp8(const moe_shape *shape, const void *x, const moe_fp8_weight *W_gate,
                 const moe_fp8_weight *W_up, const moe_fp8_weight *W_shared_gate,
                 const moe_fp8_weight *W_shared_up, void *workspace, size_t workspace_bytes,

@@ -33,7 +33,7 @@ EXPORTED = ["moe_version", "moe_status_string", "moe_workspace_bytes", "moe_forw
             "moe_forward_host", "moe_route", "moe_permute", "moe_expert_gate_up", "moe_expert_down",
             "moe_combine", "moe_workspace_region", "moe_device_status", "moe_debug_wait_timeout",
             "moe_route_noalloc", "moe_experts_forward", "moe_rmsnorm", "moe_forward_prenorm",
-            "moe_forward_fp8", "moe_expert_gate_up_fp8", "moe_expert_down_fp8"]
+            "moe_forward_fp8", "moe_expert_gate_up_fp8", "moe_expert_down_fp8", "moe_permute_fp8"]
 
 
 class MoEError(RuntimeError):
@@ -83,6 +83,8 @@ def load():
     F8 = ctypes.POINTER(MoeFp8Weight)
     lib.moe_forward_fp8.restype = I
     lib.moe_forward_fp8.argtypes = [SH, P, P, P, F8, F8, F8, F8, F8, F8] + fwd[10:]
+    lib.moe_permute_fp8.restype = I
+    lib.moe_permute_fp8.argtypes = [SH, P, P, P, SZ, P]
     lib.moe_expert_gate_up_fp8.restype = I
     lib.moe_expert_gate_up_fp8.argtypes = [SH, P, F8, F8, F8, F8, P, SZ, P]
     lib.moe_expert_down_fp8.restype = I
@@ -273,6 +275,15 @@ def moe_forward_fp8(shape, x, W_router, expert_bias, W_gate, W_up, W_down, W_sha
         _p(topk_w, torch.float32, (T, k), "topk_w"),
         _p(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream))
     _check(st, "moe_forward_fp8")
+
+
+def moe_permute_fp8(shape, topk_idx, topk_w, workspace, stream=None):
+    """The permute for the FP8 expert steps (their work lists differ from the bf16 ones)."""
+    T, k = shape.T, shape.k
+    st = load().moe_permute_fp8(ctypes.byref(shape), _p(topk_idx, torch.int32, (T, k), "topk_idx"),
+                                _p(topk_w, torch.float32, (T, k), "topk_w"),
+                                _p(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "moe_permute_fp8")
 
 
 def moe_expert_gate_up_fp8(shape, x, W_gate, W_up, W_shared_gate, W_shared_up, workspace, stream=None):
@@ -472,7 +483,7 @@ class MoELayer:
         moe_route(s, x, t["W_router"], t["expert_bias"], c.score_fn, c.norm_topk, c.route_scale,
                   self.topk_idx, self.topk_w, self.workspace, st)
         rec(1)
-        moe_permute(s, self.topk_idx, self.topk_w, self.workspace, st)
+        (moe_permute_fp8 if c.fp8 else moe_permute)(s, self.topk_idx, self.topk_w, self.workspace, st)
         rec(2)
         if c.fp8:
             moe_expert_gate_up_fp8(s, x, t["W_gate_f8"], t["W_up_f8"], t["W_shared_gate_f8"],

@@ -183,6 +183,8 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, Wt Wg, Wt Wu
   }
   copy_set(g.mapB[1], g.mapB[0]);
   g.units = reinterpret_cast<const int4*>(ws + p.units1);
+  g.plan_tag_dev = reinterpret_cast<const int*>(ws + p.nunits) + 3;
+  g.plan_tag = plan_tag(p);
   g.num_units_dev = reinterpret_cast<const int*>(ws + p.nunits);
   g.perm = reinterpret_cast<const int*>(ws + p.perm);
   g.x = x;
@@ -197,6 +199,7 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, Wt Wg, Wt Wu
   g.nbuf = (2 * p.nmax1 <= 256) ? 2 : 1;
   if (f8) {
     int raw = 0, tok = 0;
+    g.nbuf = (4 * p.nmax1 <= 256) ? 2 : 1;      // accumulators below the widened tiles
     const size_t smem = gemm_f8_smem_bytes(kModeGateUp, p.nmax1, &stages, &tok, &raw);
     g.stages = stages;
     g.tok_stages = tok;
@@ -234,6 +237,8 @@ int run_down(const Plan& p, const DeviceInfo& di, Wt Wd, Wt Wsd, char* ws, cudaS
   g.mapS[1] = g.mapS[0];
   g.mapS[3] = g.mapS[2];
   g.units = reinterpret_cast<const int4*>(ws + p.units2);
+  g.plan_tag_dev = reinterpret_cast<const int*>(ws + p.nunits) + 3;
+  g.plan_tag = plan_tag(p);
   g.num_units_dev = reinterpret_cast<const int*>(ws + p.nunits) + 1;
   g.roww = reinterpret_cast<const float*>(ws + p.roww);
   g.out_r = ws + p.Yr;
@@ -246,7 +251,7 @@ int run_down(const Plan& p, const DeviceInfo& di, Wt Wd, Wt Wsd, char* ws, cudaS
   int stages = 0;
   if (f8) {
     int raw = 0, tok = 0;
-    g.nbuf = (2 * p.nmax2 <= 256) ? 2 : 1;
+    g.nbuf = (4 * p.nmax2 <= 256) ? 2 : 1;      // accumulators below the widened tiles
     const size_t smem = gemm_f8_smem_bytes(kModeDown, p.nmax2, &stages, &tok, &raw);
     g.stages = stages;
     g.tok_stages = tok;
@@ -333,7 +338,7 @@ int check_gate_vec(const Plan& p, const void* W_shared_gate_vec) {
 
 }  // namespace
 
-int make_plan(const moe_shape* s, Plan* p) {
+int make_plan(const moe_shape* s, Plan* p, bool f8) {
   if (!s || !p) return MOE_ERR_INVALID_ARG;
   const int T = s->T, d = s->d_model, E = s->E, k = s->k, f = s->d_ff, S = s->n_shared;
   const int fs = S > 0 ? s->d_ff_shared : 0;
@@ -348,14 +353,19 @@ int make_plan(const moe_shape* s, Plan* p) {
   q.T = T; q.d = d; q.E = E; q.k = k; q.f = f; q.S = S; q.fs = fs;
   const double rows_per_expert = static_cast<double>(T) * k / E;
   q.nmax1 = pick_nmax(rows_per_expert);
-  q.nmax2 = q.nmax1;
   // Experts of 256+ rows on average: the gate/up GEMM runs on CTA pairs,
   // each CTA loading half of every token tile (runs then come in multiples of
   // 32).  Below that, and for the down GEMM (measured), the pair's cross-CTA
   // handshakes cost more than the halved token loads save.
-  q.pair1 = (q.nmax1 >= 64 && rows_per_expert >= 256.0) ? 1 : 0;
+  const int pair_bf16 = (q.nmax1 >= 64 && rows_per_expert >= 256.0) ? 1 : 0;
+  // FP8 expert weights: single CTAs, token runs of at most 128 (their
+  // accumulators share tensor memory with the widened weight tiles).  The
+  // workspace layout is the same for both weight formats.
+  if (f8 && q.nmax1 > 128) q.nmax1 = 128;
+  q.nmax2 = q.nmax1;
+  q.pair1 = f8 ? 0 : pair_bf16;
   q.pair2 = 0;
-  q.rowpad = (q.pair1 || q.pair2) ? 2 * kRowPad : kRowPad;
+  q.rowpad = pair_bf16 ? 2 * kRowPad : kRowPad;
   // Experts that fit one token run on average read each weight tile once.
   q.weights_evict_first = rows_per_expert <= 0.75 * q.nmax1 ? 1 : 0;
   q.Tp = ceil_div(T, q.rowpad) * q.rowpad;
@@ -363,6 +373,7 @@ int make_plan(const moe_shape* s, Plan* p) {
   q.nb = ceil_div(T, kPermBlock);
   q.nwbE = ceil_div(E, kTileRows);
   const int rows1 = q.pair1 ? 2 * kTileRows : kTileRows;   // weight rows per gate/up unit
+  const int ncap = q.nmax1 < 128 ? q.nmax1 : 128;          // unit-list bounds cover both formats
   const int rows2 = 2 * kTileRows;                          // weight rows per down unit
   q.nwb1 = ceil_div(f, rows1);
   q.nwb1s = S > 0 ? ceil_div(fs, rows1) : 0;
@@ -384,8 +395,9 @@ int make_plan(const moe_shape* s, Plan* p) {
   q.router_units = q.nwbE * ceil_div(q.Tp, q.nmax_r);
   q.shared_units1 = S * q.nwb1s * ceil_div(q.Tp, q.nmax1);
   q.shared_units2 = S * q.nwb2 * ceil_div(q.Tp, q.nmax2);
-  q.U1cap = q.shared_units1 + q.nwb1 * (q.Rcap / q.nmax1 + E);
-  q.U2cap = q.shared_units2 + q.nwb2 * (q.Rcap / q.nmax2 + E);
+  const int nwb1cap = ceil_div(f, kTileRows), nwb1scap = S > 0 ? ceil_div(fs, kTileRows) : 0;
+  q.U1cap = S * nwb1scap * ceil_div(q.Tp, ncap) + nwb1cap * (q.Rcap / ncap + E);
+  q.U2cap = S * q.nwb2 * ceil_div(q.Tp, ncap) + q.nwb2 * (q.Rcap / ncap + E);
 
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -630,7 +642,7 @@ int moe_forward_fp8(const moe_shape* shape, const void* x, const void* W_router,
                     float route_scale, void* out, int32_t* topk_idx, float* topk_w, void* workspace,
                     size_t workspace_bytes, moe_stream_t stream) {
   Plan p;
-  int rc = make_plan(shape, &p);
+  int rc = make_plan(shape, &p, true);
   if (rc != MOE_OK) return rc;
   if ((rc = check_route_args(x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w)) != MOE_OK)
     return rc;
@@ -647,12 +659,25 @@ int moe_forward_fp8(const moe_shape* shape, const void* x, const void* W_router,
                       topk_idx, topk_w, static_cast<char*>(workspace), as_stream(stream));
 }
 
+int moe_permute_fp8(const moe_shape* shape, const int32_t* topk_idx, const float* topk_w, void* workspace,
+                    size_t workspace_bytes, moe_stream_t stream) {
+  Plan p;
+  int rc = make_plan(shape, &p, true);
+  if (rc != MOE_OK) return rc;
+  if (!topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(topk_idx) || !aligned16(topk_w)) return MOE_ERR_UNSUPPORTED;
+  if ((rc = check_ws(p, workspace, workspace_bytes)) != MOE_OK) return rc;
+  DeviceInfo di;
+  if ((rc = check_device(&di)) != MOE_OK) return rc;
+  return launch_permute(p, topk_idx, topk_w, static_cast<char*>(workspace), as_stream(stream));
+}
+
 int moe_expert_gate_up_fp8(const moe_shape* shape, const void* x, const moe_fp8_weight* W_gate,
                            const moe_fp8_weight* W_up, const moe_fp8_weight* W_shared_gate,
                            const moe_fp8_weight* W_shared_up, void* workspace, size_t workspace_bytes,
                            moe_stream_t stream) {
   Plan p;
-  int rc = make_plan(shape, &p);
+  int rc = make_plan(shape, &p, true);
   if (rc != MOE_OK) return rc;
   if (!x || !f8_given(W_gate) || !f8_given(W_up)) return MOE_ERR_INVALID_ARG;
   if (p.S > 0 && (!f8_given(W_shared_gate) || !f8_given(W_shared_up))) return MOE_ERR_INVALID_ARG;
@@ -669,7 +694,7 @@ int moe_expert_gate_up_fp8(const moe_shape* shape, const void* x, const moe_fp8_
 int moe_expert_down_fp8(const moe_shape* shape, const moe_fp8_weight* W_down, const moe_fp8_weight* W_shared_down,
                         void* workspace, size_t workspace_bytes, moe_stream_t stream) {
   Plan p;
-  int rc = make_plan(shape, &p);
+  int rc = make_plan(shape, &p, true);
   if (rc != MOE_OK) return rc;
   if (!f8_given(W_down) || (p.S > 0 && !f8_given(W_shared_down))) return MOE_ERR_INVALID_ARG;
   if (!f8_aligned(W_down) || (p.S > 0 && !f8_aligned(W_shared_down))) return MOE_ERR_UNSUPPORTED;
@@ -752,7 +777,7 @@ int moe_device_status(const void* workspace, moe_stream_t stream) {
   uint32_t word = 0;
   if (cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
   if (word & kDevErrTimeout) return MOE_ERR_DEVICE_TIMEOUT;
-  if (word & kDevErrBadRouting) return MOE_ERR_INVALID_ARG;
+  if (word & (kDevErrBadRouting | kDevErrPlanMismatch)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 

@@ -60,6 +60,11 @@ constexpr int kMaxTokStages = 8;                     // FP8: stages of the token
 constexpr uint32_t kRawTileBytes = kTileRows * kTileK;           // 128 rows x 64 FP8 codes
 constexpr uint32_t kScaleTileBytes = kTileRows * (kTileK / 32);  // their scales: [2 blocks][128 rows]
 constexpr uint32_t kRawTile = kRawTileBytes + kScaleTileBytes;
+// FP8: widened weight tiles live in tensor memory, columns [256, 512): stage s,
+// tile a at column 256 + (2 s + a) * 32 (128 rows x 64 bf16 = 32 columns);
+// accumulators then use columns [0, 256).
+constexpr uint32_t kAColBase = 256;
+constexpr int kAStages = 4;
 constexpr int kRouterDrainKB = 2;                    // router: k-blocks accumulated in TMEM per drain
 constexpr int kRouterMaxN = 128;                     // router: tokens per unit (fp32 sums in registers)
 
@@ -161,16 +166,9 @@ __device__ __forceinline__ void fp8x16_to_bf16_cvt(const uint4 v, float sc, uint
   hi.w = fp8x2_to_bf16x2(v.w >> 16, sc);
 }
 
-// Widens one 32-code block - half h of row r of a landed FP8 tile, codes at
-// src (the row's 64 codes), scale byte s - into row r of the
-// 128-byte-swizzled bf16 tile at dst.  With threads (r, h) interleaved along
-// the warp, each 8-thread shared-memory wavefront covers 4 rows x 2 halves:
-// the stores hit 8 different bank groups and the loads 4 (2-way).
-__device__ __forceinline__ void widen_half(const uint8_t* src, uint32_t s, uint8_t* dst, int r, int h) {
-  const uint4 v0 = *reinterpret_cast<const uint4*>(src + 32 * h);
-  const uint4 v1 = *reinterpret_cast<const uint4*>(src + 32 * h + 16);
-  uint8_t* drow = dst + r * 128;
-  const int sw = r & 7;
+// Widens one 32-code block of a landed FP8 tile (its two 16-byte chunks, scale
+// byte s) into 16 packed bf16x2 registers, element pairs in K order.
+__device__ __forceinline__ void widen_block(const uint4 v0, const uint4 v1, uint32_t s, uint32_t (&o)[16]) {
   uint4 a, b, c, d;
   if (s <= 134u) {
     const uint32_t e = (s + 120u) << 7;    // bf16 bits of 2^(s-7)
@@ -181,10 +179,10 @@ __device__ __forceinline__ void widen_half(const uint8_t* src, uint32_t s, uint8
     fp8x16_to_bf16_cvt(v0, sc, a, b);
     fp8x16_to_bf16_cvt(v1, sc, c, d);
   }
-  *reinterpret_cast<uint4*>(drow + (((4 * h + 0) ^ sw) << 4)) = a;
-  *reinterpret_cast<uint4*>(drow + (((4 * h + 1) ^ sw) << 4)) = b;
-  *reinterpret_cast<uint4*>(drow + (((4 * h + 2) ^ sw) << 4)) = c;
-  *reinterpret_cast<uint4*>(drow + (((4 * h + 3) ^ sw) << 4)) = d;
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  o[8] = c.x; o[9] = c.y; o[10] = c.z; o[11] = c.w;
+  o[12] = d.x; o[13] = d.y; o[14] = d.z; o[15] = d.w;
 }
 
 // SiLU(z) = z * sigmoid(z) with the fast exponential and division; the
@@ -210,11 +208,11 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
   const int nmax = p.nmax;
   const int S = p.stages;
   const uint32_t tok_bytes = static_cast<uint32_t>(nmax) * 128u;
-  // bf16: each MMA stage holds the weight tiles and the token tile.  FP8:
-  // three rings - MMA stages of widened weight tiles (S), token tiles (TS),
-  // and the landing ring of code + scale tiles (R) - so that token loads run
-  // as far ahead as the bf16 path's, however few widened stages fit.
-  const uint32_t stage_bytes = NA * kATileBytes + (F8 ? 0u : tok_bytes);
+  // bf16: each MMA stage holds the weight tiles and the token tile in shared
+  // memory.  FP8: the MMA stages (S) hold the widened weight tiles in tensor
+  // memory, and shared memory holds two rings - token tiles (TS) and the
+  // landed code + scale tiles (R) - so both kinds of load run far ahead.
+  const uint32_t stage_bytes = F8 ? 0u : NA * kATileBytes + tok_bytes;
   const int TS = F8 ? p.tok_stages : 0;
   const int R = F8 ? p.raw_stages : 0;
   constexpr uint32_t raw_stage_bytes = NA * kRawTile;
@@ -281,7 +279,12 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   chain_wait();
-  const int num_units = (MODE == kModeRouter) ? p.num_units_host : *p.num_units_dev;
+  int num_units = (MODE == kModeRouter) ? p.num_units_host : *p.num_units_dev;
+  if (MODE != kModeRouter && *p.plan_tag_dev != p.plan_tag) {
+    // work lists built for the other weight format's plan: do nothing, report it
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(p.err, kDevErrPlanMismatch);
+    num_units = 0;
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -445,15 +448,26 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
             const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
             const uint64_t bdesc = sw128_kmajor_desc(
                 F8 ? smem_u32(tokring + static_cast<size_t>(tstage) * tok_bytes) : sbase + NA * kATileBytes);
-            uint64_t adesc[NA];
+            if constexpr (F8) {
+              const uint32_t acol = tmem_base + kAColBase + static_cast<uint32_t>(stage * NA * 32);
 #pragma unroll
-            for (int a = 0; a < NA; ++a) adesc[a] = sw128_kmajor_desc(sbase + a * kATileBytes);
+              for (int ks = 0; ks < kTileK / 16; ++ks) {
 #pragma unroll
-            for (int ks = 0; ks < kTileK / 16; ++ks) {
+                for (int a = 0; a < NA; ++a)
+                  tc_mma_bf16_ta(dcol + static_cast<uint32_t>(a * nmax), acol + static_cast<uint32_t>(a * 32 + ks * 8),
+                                 bdesc + 2u * ks, idesc, (kb | ks) != 0 ? 1u : 0u);
+              }
+            } else {
+              uint64_t adesc[NA];
 #pragma unroll
-              for (int a = 0; a < NA; ++a)
-                tc_mma_bf16(dcol + static_cast<uint32_t>(a * nmax), adesc[a] + 2u * ks, bdesc + 2u * ks,
-                            idesc, (kb | ks) != 0 ? 1u : 0u);
+              for (int a = 0; a < NA; ++a) adesc[a] = sw128_kmajor_desc(sbase + a * kATileBytes);
+#pragma unroll
+              for (int ks = 0; ks < kTileK / 16; ++ks) {
+#pragma unroll
+                for (int a = 0; a < NA; ++a)
+                  tc_mma_bf16(dcol + static_cast<uint32_t>(a * nmax), adesc[a] + 2u * ks, bdesc + 2u * ks,
+                              idesc, (kb | ks) != 0 ? 1u : 0u);
+              }
             }
             any = true;
             tc_commit(&empty[stage]);
@@ -483,12 +497,17 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
     __syncwarp();
   } else if (F8 && warp >= kConvBase) {
     // ------------------------------------------------------------ FP8 -> bf16
-    // Thread c widens block (c & 1) of row (c >> 1) of every landed code
-    // tile into the MMA stage.
-    const int c = threadIdx.x - 32 * kConvBase;
-    const int crow = c >> 1, chalf = c & 1;
+    // Warp w may access tensor-memory lanes 32 (w % 4) .. + 31: its lane l
+    // widens 32-code block h of weight row r = 32 (w % 4) + l of every landed
+    // code tile into the MMA stage's tile in tensor memory; the first four
+    // converter warps take h = 0, the next four h = 1.
+    const int cq = warp & 3;
+    const int crow = 32 * cq + lane;
+    const int chalf = (warp - kConvBase) >> 2;
+    const uint32_t tlane = static_cast<uint32_t>(32 * cq) << 16;
     int rs = 0, ms = 0;              // landing-ring and MMA-ring positions
     uint32_t rph = 0, mph = 0;
+    int pms = -1;                    // MMA stage written but not yet published
     bool ok = true;
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
       const Unit un = get_unit<MODE>(p, u);
@@ -507,20 +526,36 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
           ok = false;
           break;
         }
-        uint8_t* sb = smem + static_cast<size_t>(ms) * stage_bytes;
+        // Codes and scales of both tiles into registers; the landed stage is
+        // then free for the producer.
         const uint8_t* rt = raw + static_cast<size_t>(rs) * raw_stage_bytes;
+        uint4 cv[NA][2];
+        uint32_t sc[NA];
 #pragma unroll
         for (int a = 0; a < NA; ++a) {
           const uint8_t* q = rt + a * kRawTile;
-          widen_half(q + crow * kTileK, q[kRawTileBytes + chalf * kTileRows + crow], sb + a * kATileBytes, crow,
-                     chalf);
+          cv[a][0] = *reinterpret_cast<const uint4*>(q + crow * kTileK + 32 * chalf);
+          cv[a][1] = *reinterpret_cast<const uint4*>(q + crow * kTileK + 32 * chalf + 16);
+          sc[a] = q[kRawTileBytes + chalf * kTileRows + crow];
         }
-        fence_proxy_async_smem();      // generic-proxy stores -> tensor-core reads
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&raw_empty[rs]);
-          mbar_arrive(&full[ms]);
+        if (lane == 0) mbar_arrive(&raw_empty[rs]);
+        // The previous k-block's tensor-memory stores have had this block's
+        // waits and loads to complete in: publish that stage now.
+        if (pms >= 0) {
+          tmem_st_wait();
+          tc_fence_before();           // tensor-memory stores -> the MMA issuer
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[pms]);
         }
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+          uint32_t w16[16];
+          widen_block(cv[a][0], cv[a][1], sc[a], w16);
+          tmem_st_32x32b_x16(tmem_base + tlane + kAColBase + static_cast<uint32_t>((ms * NA + a) * 32 + 16 * chalf),
+                             w16);
+        }
+        pms = ms;
         if (++rs == R) {
           rs = 0;
           rph ^= 1u;
@@ -530,6 +565,12 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
           mph ^= 1u;
         }
       }
+    }
+    if (pms >= 0) {
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[pms]);
     }
   } else if (F8 && MODE == kModeDown && warp == kTokWarp) {
     // ------------------------------------------------------------ FP8 down: token rows
@@ -896,7 +937,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   chain_wait();
-  const int num_units = *p.num_units_dev;
+  int num_units = *p.num_units_dev;
+  if (*p.plan_tag_dev != p.plan_tag) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(p.err, kDevErrPlanMismatch);
+    num_units = 0;
+  }
   const uint32_t full_leader = mapa_shared(smem_u32(full), 0);     // + 8 * stage
   const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0); // + 8 * buf
 
@@ -1232,13 +1277,13 @@ int launch_gemm_pair(int mode, const GemmParams& prm, int grid, size_t smem, cud
 
 size_t gemm_f8_smem_bytes(int mode, int nmax, int* stages, int* tok_stages, int* raw_stages) {
   const int NA = 2;   // gate/up and down both stage two weight tiles
-  const size_t stage_bytes = NA * static_cast<size_t>(kATileBytes);
+  const size_t stage_bytes = 0;   // widened tiles live in tensor memory
   const size_t tok_bytes = static_cast<size_t>(nmax) * 128;
   const size_t raw_stage = NA * static_cast<size_t>(kRawTile);
   const size_t fixed = kSmemAlign + kEpiBytes + kSmemTail;
   const size_t budget = 232448;
   (void)mode;
-  const int s = 2;    // the converters fill one MMA stage while the tensor cores read the other
+  const int s = kAStages;
   int ts = static_cast<int>(65536 / tok_bytes);   // 64 KB of token tiles
   if (ts < 2) ts = 2;
   if (ts > kMaxTokStages) ts = kMaxTokStages;
@@ -1271,8 +1316,9 @@ static int launch_mode(const GemmParams& prm, int grid, size_t smem, cudaStream_
 int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st, bool f8) {
   if (grid < 1) return MOE_OK;
   if (f8) {
-    if (prm.raw_stages < 2 || prm.raw_stages > kMaxRawStages || prm.stages != 2 || prm.tok_stages < 2 ||
-        prm.tok_stages > kMaxTokStages)
+    // the accumulators must fit below the widened tiles' columns
+    if (prm.raw_stages < 2 || prm.raw_stages > kMaxRawStages || prm.stages != kAStages || prm.tok_stages < 2 ||
+        prm.tok_stages > kMaxTokStages || prm.nmax > 128 || 2 * prm.nmax * prm.nbuf > static_cast<int>(kAColBase))
       return MOE_ERR_INVALID_ARG;
     switch (mode) {
       case kModeGateUp: return launch_mode<kModeGateUp, true>(prm, grid, smem, st);

@@ -79,7 +79,10 @@ struct Plan {
 };
 
 // Fills `p` for `s`; returns MOE_OK or MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED.
-int make_plan(const moe_shape* s, Plan* p);
+int make_plan(const moe_shape* s, Plan* p, bool f8 = false);
+// Tag of the work-list layout a plan produces (token-run length, CTA pairs);
+// the permute stores it beside the lists and the expert GEMMs check it.
+inline int plan_tag(const Plan& p) { return p.nmax1 | (p.pair1 << 12) | (1 << 16); }
 
 // Per-device facts, looked up once per device.
 struct DeviceInfo {
@@ -113,6 +116,8 @@ struct GemmParams {
   // tiles of 128 rows x 2 blocks); raw_stages = depth of the landing ring
   CUtensorMap mapS[4];
   int raw_stages, tok_stages;
+  const int* plan_tag_dev;  // expert GEMMs: the tag the permute stored
+  int plan_tag;             // the tag this launch's plan expects
 };
 
 int launch_gemm(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st, bool f8 = false);

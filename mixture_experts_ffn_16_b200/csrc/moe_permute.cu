@@ -124,6 +124,7 @@ struct ScanArgs {
   int nb, E, T, Tp, rowpad;
   int nmax1, nmax2, nwb1, nwb1s, nwb2, S;
   int shared_units1, shared_units2;
+  int plan_tag;
 };
 
 __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) {
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) 
     a.nunits[0] = a.shared_units1 + tot1;
     a.nunits[1] = a.shared_units2 + tot2;
     a.nunits[2] = tot_rows;
-    a.nunits[3] = 0;
+    a.nunits[3] = a.plan_tag;   // which work-list layout this is (checked by the expert GEMMs)
   }
 }
 
@@ -283,6 +284,7 @@ int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, 
   a.S = p.S;
   a.shared_units1 = p.shared_units1;
   a.shared_units2 = p.shared_units2;
+  a.plan_tag = plan_tag(p);
   if (launch_chained(permute_scan_kernel, dim3(1), dim3(kScanThreads), 0, st, a) != cudaSuccess) return MOE_ERR_CUDA;
 
   return launch_chained(permute_scatter_kernel, dim3(p.nb), dim3(kPermBlock), msmem, st, topk_idx, topk_w, p.T, p.E,

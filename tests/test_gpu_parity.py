@@ -336,3 +336,25 @@ def test_fp8_widening_edge_codes(oracle_mod, kind):
     out, idx, w, _ = run_gpu(cfg, inp)
     rep = check_parity(oracle_mod, cfg, _fp8_host_args(oracle_mod, inp), out, idx, w)
     print(cfg.name, rep)
+
+
+def test_fp8_steps_refuse_bf16_work_lists(oracle_mod):
+    """With large experts the bf16 plan uses 256-token runs and CTA pairs, the
+    FP8 plan 128-token runs: an FP8 expert step fed bf16 work lists must do
+    nothing and report MOE_ERR_INVALID_ARG; the FP8 permute then fixes it."""
+    _need_gpu()
+    cfg = [c for c in FP8 if c.name == "fp8_many_rows_gated"][0]
+    inp = make_inputs(cfg, device="cuda")
+    layer = api.MoELayer(cfg, inp)
+    s, t = layer.shape, inp
+    api.moe_route(s, t["x"], t["W_router"], t["expert_bias"], cfg.score_fn, cfg.norm_topk, cfg.route_scale,
+                  layer.topk_idx, layer.topk_w, layer.workspace)
+    api.moe_permute(s, layer.topk_idx, layer.topk_w, layer.workspace)
+    api.moe_expert_gate_up_fp8(s, t["x"], t["W_gate_f8"], t["W_up_f8"], t["W_shared_gate_f8"],
+                               t["W_shared_up_f8"], layer.workspace)
+    assert api.moe_device_status(layer.workspace) == api.MOE_ERR_INVALID_ARG
+    out1 = layer()[0].clone()                      # moe_forward_fp8 clears the error word
+    assert api.moe_device_status(layer.workspace) == api.MOE_OK
+    out2 = layer.steps()[0].clone()
+    assert api.moe_device_status(layer.workspace) == api.MOE_OK
+    assert torch.equal(out1, out2)
