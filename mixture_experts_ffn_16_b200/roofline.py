@@ -77,9 +77,9 @@ def block_cost(cfg, touched=None):
 # the ncu captures summarised in profiles/gemm_<workload>.md.  A figure is
 # valid only while the GEMM source is the one that was captured (sha256 prefix).
 NCU_TRAFFIC = {
-    ("prefill_softmax", "route"): (17.9e6, "9086017a9f5ca9dc"),
-    ("prefill_softmax", "gate_up"): (1209.6e6, "9086017a9f5ca9dc"),
-    ("prefill_softmax", "down"): (719.3e6, "9086017a9f5ca9dc"),
+    ("prefill_softmax", "route"): (17.9e6, "20c1b7a09bf53c47"),
+    ("prefill_softmax", "gate_up"): (1109.8e6, "20c1b7a09bf53c47"),
+    ("prefill_softmax", "down"): (746.4e6, "20c1b7a09bf53c47"),
 }
 
 
