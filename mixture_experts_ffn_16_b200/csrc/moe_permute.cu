@@ -8,7 +8,8 @@
 //             count; then exclusive scans over experts of the padded segment
 //             sizes and of the GEMM work-unit counts; writes the work lists
 //             and fills the padding rows.
-//   scatter : recomputes the masks; a (token, slot) pair's row is
+//   scatter : recomputes the masks (each of the ceil(k/2) CTAs of a block
+//             places two slots of its tokens); a (token, slot) pair's row is
 //             segment start + block offset + popcount of the lower lanes of
 //             the lower warps and of its own warp: rows inside an expert are in
 //             ascending token order, so the layout is deterministic.
@@ -28,6 +29,7 @@ namespace {
 
 constexpr int kWarps = kPermBlock / 32;
 constexpr int kScanThreads = 1024;
+constexpr int kScatterSlots = 2;   // (token, slot) pairs per scatter thread
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
@@ -225,7 +227,10 @@ permute_scatter_kernel(const int32_t* __restrict__ topk_idx, const float* __rest
   if (t >= T) return;
   const int w = threadIdx.x >> 5;
   const uint32_t lt = lanemask_lt();
-  for (int j = 0; j < k; ++j) {
+  // CTAs (x, y) share block x's masks; CTA y places slots [y s, y s + s).
+  const int j0 = blockIdx.y * kScatterSlots;
+  const int j1 = min(k, j0 + kScatterSlots);
+  for (int j = j0; j < j1; ++j) {
     const size_t tj = static_cast<size_t>(t) * k + j;
     const int e = topk_idx[tj];
     if (e < 0 || e >= E) {
@@ -287,7 +292,8 @@ int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, 
   a.plan_tag = plan_tag(p);
   if (launch_chained(permute_scan_kernel, dim3(1), dim3(kScanThreads), 0, st, a) != cudaSuccess) return MOE_ERR_CUDA;
 
-  return launch_chained(permute_scatter_kernel, dim3(p.nb), dim3(kPermBlock), msmem, st, topk_idx, topk_w, p.T, p.E,
+  return launch_chained(permute_scatter_kernel, dim3(p.nb, (p.k + kScatterSlots - 1) / kScatterSlots),
+                        dim3(kPermBlock), msmem, st, topk_idx, topk_w, p.T, p.E,
                         p.k, blkcnt, a.roff, a.perm, a.roww, reinterpret_cast<int32_t*>(ws + p.inv),
                         err) == cudaSuccess
              ? MOE_OK

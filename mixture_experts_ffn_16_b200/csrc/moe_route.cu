@@ -3,7 +3,8 @@
 // One warp per token reads the token's fp32 logits (written by the router
 // GEMM), forms the scores and selection keys in registers, and picks the k
 // largest keys by k rounds of a warp-wide arg-max (ties go to the lower expert
-// index, matching a stable descending sort).
+// index, matching a stable descending sort); each round reduces the lanes'
+// best keys with two warp reductions.
 //
 //   softmax       : key = logit (same order as the softmax probability);
 //                   w_j = exp(l_j - l_max) / (norm ? sum over picks : sum over all E)
@@ -87,15 +88,13 @@ topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, in
         bi = e;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (better(ok, oi, bk, bi)) {
-        bk = ok;
-        bi = oi;
-      }
-    }
+    // Warp arg-max in two reductions: the largest key (as an order-preserving
+    // unsigned integer), then the lowest expert index among the lanes that
+    // hold it.
+    const uint32_t ub = __float_as_uint(bk + 0.0f);   // -0 -> +0: equal keys stay equal
+    const uint32_t uk = (ub & 0x80000000u) ? ~ub : (ub | 0x80000000u);
+    const uint32_t umax = __reduce_max_sync(0xffffffffu, uk);
+    bi = static_cast<int>(__reduce_min_sync(0xffffffffu, uk == umax ? static_cast<uint32_t>(bi) : 0x7fffffffu));
     // Remove the winner (its owner lane), record it in lane j.
 #pragma unroll
     for (int i = 0; i < NPL; ++i)
