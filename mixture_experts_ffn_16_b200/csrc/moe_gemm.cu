@@ -11,15 +11,20 @@
 // (n a multiple of 16), so an expert with few tokens costs n/16 MMA columns,
 // not a padded 128-row tile.
 //
-//   warp 0      TMA producer: weight tiles by 3-D tiled loads, token rows by
-//               tile::gather4 loads (4 arbitrary rows per instruction, no
-//               permuted copy of x is ever made), into a ring of stages.
+//   warp 0      TMA producer: weight tiles by 3-D tiled loads (and, for the
+//               router and the down GEMM, the unit's contiguous token rows)
+//               into a ring of stages.
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer; fp32
 //               accumulators in tensor memory (gate and up side by side for
 //               the gate/up GEMM), double-buffered when they fit.
-//   warps 2..5  epilogue: tcgen05.ld -> fp32 math (SiLU*, weight scale) ->
-//               bf16 -> transpose through shared memory -> 16-byte stores of
-//               whole row segments.
+//   epilogue    4 (router) or 8 warps: tcgen05.ld -> fp32 math (SiLU*, weight
+//               scale) -> bf16 -> transpose through shared memory -> 16-byte
+//               stores of whole row segments.
+//   gather      gate/up: 4 warps copy the unit's token rows of x (by perm) with
+//               cp.async straight into the swizzled tile; no permuted copy of
+//               x is ever made.
+//   FP8 forms   block-scaled FP8 weights: converter warps widen landed FP8
+//               tiles into tensor memory (see moe_gemm_kernel<MODE, true>).
 //
 // All waits are bounded (see mbar_wait); a block that gives up records the
 // timeout in the workspace error word, drains its own copies and MMAs, frees
