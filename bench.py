@@ -285,7 +285,10 @@ def run_ours(args, cfg):
     if st != api.MOE_OK:
         raise RuntimeError(f"device status after warm-up: {api.status_string(st)}")
     idx_host = (ext_idx if external else layer.topk_idx).cpu().numpy()
-    touched = int((np.bincount(idx_host.ravel(), minlength=cfg.E) > 0).sum())
+    load = np.bincount(idx_host.ravel(), minlength=cfg.E)
+    touched = int((load > 0).sum())
+    expert_load = {"max": int(load.max()), "median": float(np.median(load)), "min": int(load.min()),
+                   "empty": int((load == 0).sum())}
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
@@ -302,6 +305,7 @@ def run_ours(args, cfg):
         for j, name in enumerate(STAGES):
             stage_ms[name] += ev[j].elapsed_time(ev[j + 1])
     stage_avg_us = {n: 1e3 * v / K for n, v in stage_ms.items()}
+    step_median_ms = float(np.median([ev[0].elapsed_time(ev[5]) for ev in evs]))
     elapsed_ms = max_over_ranks(elapsed_ms, world)
     st = api.moe_device_status(layer.workspace, stream)
     if st != api.MOE_OK:
@@ -398,11 +402,12 @@ def run_ours(args, cfg):
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "warmup": args.warmup, "ms_per_step": ms_step, "ms_per_step_median": step_median_ms,
+                "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) x, N(0,0.02) weights)",
                 "config": {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "E": cfg.E, "k": cfg.k,
                            "d_ff": cfg.f, "n_shared": cfg.S, "d_ff_shared": cfg.fs, "score_fn": cfg.score_fn,
-                           "norm_topk": cfg.norm_topk, "touched_experts": touched,
+                           "norm_topk": cfg.norm_topk, "touched_experts": touched, "expert_load": expert_load,
                            "variant": args.variant or "base",
                            "expert_weights": "fp8 e4m3 + ue8m0 scale per 32" if cfg.fp8 else "bf16",
                            "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (
