@@ -273,7 +273,10 @@ MOE_API int moe_experts_forward(const moe_shape *shape, const void *x, const int
                                 void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* Introspection of the workspace layout, for tests and debugging.  Regions:
- *   MOE_WS_LOGITS   fp32 [T,E]   router logits (after moe_route)
+ *   MOE_WS_LOGITS   fp32 [P,T,E] router logits (after moe_route) as P partial
+ *                                sums over slices of d, added in slice order
+ *                                (P = 1 unless the batch is too small to
+ *                                fill the GPU with token runs alone)
  *   MOE_WS_COUNTS   int32 [E]    tokens per expert (after moe_permute)
  *   MOE_WS_OFFSETS  int32 [E+1]  first row of each expert's segment; segments
  *                                are padded to 16 rows; [E] = total rows

@@ -151,6 +151,8 @@ int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_
   g.T = p.T; g.Tp = p.Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
   g.nmax = p.nmax_r;
   g.router_nwb = p.nwbE;
+  g.router_split = p.router_split;
+  g.router_kbs = p.router_kbs;
   g.timeout_ns = kWaitTimeoutNs;
   int stages = 0;
   const size_t smem = gemm_smem_bytes(kModeRouter, p.nmax_r, &stages);
@@ -159,8 +161,8 @@ int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_
   const int grid = p.router_units < di.sms ? p.router_units : di.sms;
   int rc = launch_gemm(kModeRouter, g, grid, smem, st);
   if (rc != MOE_OK) return rc;
-  return launch_topk(reinterpret_cast<const float*>(ws + p.logits), bias, p.T, p.E, p.k, score_fn, norm_topk,
-                     route_scale, topk_idx, topk_w, st);
+  return launch_topk(reinterpret_cast<const float*>(ws + p.logits), p.router_split, bias, p.T, p.E, p.k, score_fn,
+                     norm_topk, route_scale, topk_idx, topk_w, st);
 }
 
 int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, Wt Wg, Wt Wu, Wt Wsg, Wt Wsu, char* ws,
@@ -392,7 +394,22 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
       }
     }
   }
-  q.router_units = q.nwbE * ceil_div(q.Tp, q.nmax_r);
+  // Too few runs to fill the SMs (decode-sized batches): split K as well, each
+  // slice writing its own partial logits, summed in slice order by top-k.
+  {
+    const int base = q.nwbE * ceil_div(q.Tp, q.nmax_r);
+    const int KB = d / kTileK;
+    int split = 1;
+    if (base < 74) {
+      split = 148 / base;
+      if (split > kMaxRouterSplit) split = kMaxRouterSplit;
+      if (split > KB) split = KB;
+      if (split < 1) split = 1;
+    }
+    q.router_kbs = ceil_div(KB, split);
+    q.router_split = ceil_div(KB, q.router_kbs);   // no empty slice
+    q.router_units = base * q.router_split;
+  }
   q.shared_units1 = S * q.nwb1s * ceil_div(q.Tp, q.nmax1);
   q.shared_units2 = S * q.nwb2 * ceil_div(q.Tp, q.nmax2);
   const int nwb1cap = ceil_div(f, kTileRows), nwb1scap = S > 0 ? ceil_div(fs, kTileRows) : 0;
@@ -407,7 +424,7 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
   };
   q.err = take(16);
   q.nunits = take(16);
-  q.logits = take(static_cast<size_t>(T) * E * 4);
+  q.logits = take(static_cast<size_t>(q.router_split) * T * E * 4);
   q.blkcnt = take(static_cast<size_t>(q.nb) * E * 4);
   q.counts = take(static_cast<size_t>(E) * 4);
   q.roff = take(static_cast<size_t>(E + 1) * 4);
@@ -754,7 +771,7 @@ int moe_workspace_region(const moe_shape* shape, int region, size_t* offset, siz
   if (make_plan(shape, &p) != MOE_OK) return MOE_ERR_INVALID_ARG;
   const size_t T = p.T, E = p.E, k = p.k, R = p.Rcap, S = p.S, Tp = p.Tp;
   switch (region) {
-    case MOE_WS_LOGITS: *offset = p.logits; *bytes = T * E * 4; break;
+    case MOE_WS_LOGITS: *offset = p.logits; *bytes = static_cast<size_t>(p.router_split) * T * E * 4; break;
     case MOE_WS_COUNTS: *offset = p.counts; *bytes = E * 4; break;
     case MOE_WS_OFFSETS: *offset = p.roff; *bytes = (E + 1) * 4; break;
     case MOE_WS_PERM: *offset = p.perm; *bytes = R * 4; break;
@@ -840,8 +857,17 @@ extern "C" int moe_route_noalloc(const moe_shape* shape, const void* x, const vo
   if (rc != MOE_OK) return rc;
   if ((rc = check_route_args(x, W_router, expert_bias, score_fn, norm_topk, route_scale, topk_idx, topk_w)) != MOE_OK)
     return rc;
-  if (static_cast<size_t>(p.T) * static_cast<size_t>(p.E) * sizeof(float) > kNoAllocLogitBytes)
-    return MOE_ERR_SCRATCH_LIMIT;
+  const size_t slice_bytes = static_cast<size_t>(p.T) * static_cast<size_t>(p.E) * sizeof(float);
+  if (slice_bytes > kNoAllocLogitBytes) return MOE_ERR_SCRATCH_LIMIT;
+  if (static_cast<size_t>(p.router_split) * slice_bytes > kNoAllocLogitBytes) {
+    // fewer K slices, so that their partial logits fit the scratch
+    const int KB = p.d / kTileK;
+    const int base = p.router_units / p.router_split;
+    const int split = static_cast<int>(kNoAllocLogitBytes / slice_bytes);
+    p.router_kbs = ceil_div(KB, split);
+    p.router_split = ceil_div(KB, p.router_kbs);
+    p.router_units = base * p.router_split;
+  }
   DeviceInfo di;
   if ((rc = check_device(&di)) != MOE_OK) return rc;
   char* scratch = nullptr;
@@ -863,6 +889,8 @@ extern "C" int moe_route_noalloc(const moe_shape* shape, const void* x, const vo
   g.T = p.T; g.Tp = p.Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
   g.nmax = p.nmax_r;
   g.router_nwb = p.nwbE;
+  g.router_split = p.router_split;
+  g.router_kbs = p.router_kbs;
   g.timeout_ns = kWaitTimeoutNs;
   int stages = 0;
   const size_t smem = gemm_smem_bytes(kModeRouter, p.nmax_r, &stages);
@@ -870,5 +898,6 @@ extern "C" int moe_route_noalloc(const moe_shape* shape, const void* x, const vo
   g.nbuf = 512 / p.nmax_r < 8 ? 512 / p.nmax_r : 8;
   const int grid = p.router_units < di.sms ? p.router_units : di.sms;
   if ((rc = launch_gemm(kModeRouter, g, grid, smem, st)) != MOE_OK) return rc;
-  return launch_topk(logits, expert_bias, p.T, p.E, p.k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
+  return launch_topk(logits, p.router_split, expert_bias, p.T, p.E, p.k, score_fn, norm_topk, route_scale, topk_idx,
+                     topk_w, st);
 }

@@ -81,9 +81,11 @@ template <int MODE>
 __device__ __forceinline__ Unit get_unit(const GemmParams& p, int u) {
   Unit un;
   if (MODE == kModeRouter) {
-    const int chunk = u / p.router_nwb;
-    un.g = 0;
-    un.wb = u - chunk * p.router_nwb;
+    // router: g = the unit's slice of K (split-K when there are few units)
+    const int v = u / p.router_split;
+    const int chunk = v / p.router_nwb;
+    un.g = u - v * p.router_split;
+    un.wb = v - chunk * p.router_nwb;
     un.row0 = chunk * p.nmax;
     un.n = min(p.nmax, p.Tp - un.row0);
   } else {
@@ -313,6 +315,9 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
       const int sidx = sh ? un.g - p.E : 0;
       const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
       const int KB = K / kTileK;
+      // router: this unit's k-blocks [kb0, kb1); the expert GEMMs: all of K
+      const int kb0 = (MODE == kModeRouter) ? un.g * p.router_kbs : 0;
+      const int kb1 = (MODE == kModeRouter) ? min(KB, kb0 + p.router_kbs) : KB;
       const CUtensorMap* mA = &p.mapA[sh ? 2 : 0];
       const CUtensorMap* mB = p.mapB[(MODE == kModeDown && sh) ? 1 : 0];
       const int a_c2 = (MODE == kModeRouter) ? 0 : (sh ? sidx : un.g);
@@ -323,7 +328,7 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
           NA * kATileBytes + (MODE == kModeGateUp ? 0u : static_cast<uint32_t>(un.n) * 128u);
       int got = 1;
       if (lane == 0) {
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&pempty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
             got = 0;
             break;
@@ -390,10 +395,12 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
           const Unit un = get_unit<MODE>(p, u);
           const int KB = p.d / kTileK;
+          const int kb0 = un.g * p.router_kbs;
+          const int kb1 = min(KB, kb0 + p.router_kbs);
           const uint32_t idesc = idesc_bf16_f32(kTileRows, un.n);
           uint32_t dcol = tmem_base;
-          for (int kb = 0; kb < KB; ++kb) {
-            const int sub = kb % kRouterDrainKB;
+          for (int kb = kb0; kb < kb1; ++kb) {
+            const int sub = (kb - kb0) % kRouterDrainKB;
             const int buf = static_cast<int>(dc % static_cast<uint32_t>(p.nbuf));
             if (sub == 0) {
               const uint32_t bpar = (dc / static_cast<uint32_t>(p.nbuf)) & 1u;
@@ -421,7 +428,7 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
               stage = 0;
               phase ^= 1u;
             }
-            if (sub == kRouterDrainKB - 1 || kb == KB - 1) {
+            if (sub == kRouterDrainKB - 1 || kb == kb1 - 1) {
               tc_commit(&tfull[buf]);
               ++dc;
             }
@@ -683,7 +690,10 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
         const Unit un = get_unit<MODE>(p, u);
         const int KB = p.d / kTileK;
-        const int nd = (KB + kRouterDrainKB - 1) / kRouterDrainKB;
+        const int kb0 = un.g * p.router_kbs;
+        const int nkb = min(KB, kb0 + p.router_kbs) - kb0;
+        const int nd = (nkb + kRouterDrainKB - 1) / kRouterDrainKB;
+        float* const lbase = reinterpret_cast<float*>(p.out_r) + static_cast<size_t>(un.g) * p.T * p.E;
         const int feat0 = un.wb * kTileRows + 32 * q;
         const bool live = feat0 < p.E;
         float acc[kRouterMaxN];
@@ -740,7 +750,7 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
               const int t = un.row0 + 16 * c + tok;
               const int e = feat0 + part * 4;
               if (t < p.T) {
-                float* dst = reinterpret_cast<float*>(p.out_r) + static_cast<size_t>(t) * p.E + e;
+                float* dst = lbase + static_cast<size_t>(t) * p.E + e;
                 const float4 vv = *reinterpret_cast<const float4*>(sf + tok * 32 + part * 4);
                 if ((p.E & 3) == 0 && e + 3 < p.E) {
                   *reinterpret_cast<float4*>(dst) = vv;

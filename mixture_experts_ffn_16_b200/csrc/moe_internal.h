@@ -14,6 +14,7 @@ namespace moe {
 
 constexpr int kMaxE = 2048;
 constexpr int kMaxK = 32;
+constexpr int kMaxRouterSplit = 16;   // K slices of the router GEMM for small batches
 constexpr int kMaxShared = 8;
 constexpr int kTileRows = 128;     // weight rows per GEMM work unit (MMA M)
 constexpr int kTileK = 64;         // bf16 elements per 128-byte swizzled row
@@ -70,6 +71,8 @@ struct Plan {
   int nwb1s;       // the same for fs
   int nwb2;        // weight blocks of d per down unit: 256 rows
   int router_units;
+  int router_split;  // router K slices (partial logits summed by the top-k kernel in slice order)
+  int router_kbs;    // k-blocks per slice
   int U1cap, U2cap;
   int shared_units1, shared_units2;
   // region offsets (bytes)
@@ -109,6 +112,7 @@ struct GemmParams {
   uint32_t* err;
   int T, Tp, E, d, f, fs;
   int nmax, stages, nbuf, router_nwb;
+  int router_split, router_kbs;   // router: K slices per token run, k-blocks per slice
   uint64_t timeout_ns;
   int weights_evict_first;  // 1: each weight tile is read by one unit (experts fit one token run)
   // block-scaled FP8 expert weights: mapA are then the code tensors (uint8,
@@ -128,9 +132,8 @@ size_t gemm_f8_smem_bytes(int mode, int nmax, int* stages, int* tok_stages, int*
 int launch_gemm_pair(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st);
 size_t gemm_pair_smem_bytes(int mode, int nmax, int* stages);
 
-int launch_topk(const float* logits, const float* bias, int T, int E, int k, int score_fn,
-                int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w,
-                cudaStream_t st);
+int launch_topk(const float* logits, int nsplit, const float* bias, int T, int E, int k, int score_fn,
+                int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w, cudaStream_t st);
 
 int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, char* ws,
                    cudaStream_t st);

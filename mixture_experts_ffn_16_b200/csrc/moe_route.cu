@@ -1,7 +1,8 @@
 // moe_route.cu - scoring, top-k selection and combine weights (step a2).
 //
 // One warp per token reads the token's fp32 logits (written by the router
-// GEMM), forms the scores and selection keys in registers, and picks the k
+// GEMM; for small batches as partial sums over slices of d, added here in
+// slice order), forms the scores and selection keys in registers, and picks the k
 // largest keys by k rounds of a warp-wide arg-max (ties go to the lower expert
 // index, matching a stable descending sort); each round reduces the lanes'
 // best keys with two warp reductions.
@@ -38,7 +39,7 @@ __device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
 
 template <int NPL>   // keys per lane: E <= 32 * NPL
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
-topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
+topk_kernel(const float* __restrict__ logits, int nsplit, const float* __restrict__ bias, int T, int E, int k,
             int score_fn, int norm_topk, float route_scale, int32_t* __restrict__ topk_idx,
             float* __restrict__ topk_w) {
   chain_wait();
@@ -46,6 +47,13 @@ topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, in
   const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   if (t >= T) return;
   const float* row = logits + static_cast<size_t>(t) * E;
+  const size_t slice = static_cast<size_t>(T) * E;
+  // logit = the sum of the K slices' partial logits, in slice order
+  auto logit_of = [&](int e) {
+    float l = row[e];
+    for (int s = 1; s < nsplit; ++s) l += row[s * slice + e];
+    return l;
+  };
   const bool use_bias = (bias != nullptr) && (score_fn != MOE_SCORE_SOFTMAX);
 
   float key[NPL];
@@ -55,7 +63,7 @@ topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, in
     const int e = lane + 32 * i;
     float kv = -INFINITY;
     if (e < E) {
-      const float l = row[e];
+      const float l = logit_of(e);
       lmax = fmaxf(lmax, l);
       kv = (score_fn == MOE_SCORE_SOFTMAX) ? l : score_of(l, score_fn) + (use_bias ? bias[e] : 0.0f);
     }
@@ -106,7 +114,7 @@ topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, in
 
   float s = 0.0f;
   if (lane < k) {
-    const float l = row[my_idx];
+    const float l = logit_of(my_idx);
     s = (score_fn == MOE_SCORE_SOFTMAX) ? expf(l - lmax) : score_of(l, score_fn);
   }
   float denom;
@@ -125,27 +133,28 @@ topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, in
 }
 
 template <int NPL>
-int launch_npl(const float* logits, const float* bias, int T, int E, int k, int fn, int norm,
+int launch_npl(const float* logits, int nsplit, const float* bias, int T, int E, int k, int fn, int norm,
                float scale, int32_t* idx, float* w, cudaStream_t st) {
   const int grid = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  return launch_chained(topk_kernel<NPL>, dim3(grid), dim3(kWarpsPerBlock * 32), 0, st, logits, bias, T, E, k, fn,
-                        norm, scale, idx, w) == cudaSuccess
+  return launch_chained(topk_kernel<NPL>, dim3(grid), dim3(kWarpsPerBlock * 32), 0, st, logits, nsplit, bias, T, E,
+                        k, fn, norm, scale, idx, w) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
 
 }  // namespace
 
-int launch_topk(const float* logits, const float* bias, int T, int E, int k, int score_fn,
-                int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w,
-                cudaStream_t st) {
-  if (E <= 32) return launch_npl<1>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
-  if (E <= 64) return launch_npl<2>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
-  if (E <= 128) return launch_npl<4>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
-  if (E <= 256) return launch_npl<8>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
-  if (E <= 512) return launch_npl<16>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
-  if (E <= 1024) return launch_npl<32>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
-  return launch_npl<64>(logits, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st);
+int launch_topk(const float* logits, int nsplit, const float* bias, int T, int E, int k, int score_fn,
+                int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+#define MOE_TOPK(NPL) launch_npl<NPL>(logits, nsplit, bias, T, E, k, score_fn, norm_topk, route_scale, topk_idx, topk_w, st)
+  if (E <= 32) return MOE_TOPK(1);
+  if (E <= 64) return MOE_TOPK(2);
+  if (E <= 128) return MOE_TOPK(4);
+  if (E <= 256) return MOE_TOPK(8);
+  if (E <= 512) return MOE_TOPK(16);
+  if (E <= 1024) return MOE_TOPK(32);
+  return MOE_TOPK(64);
+#undef MOE_TOPK
 }
 
 }  // namespace moe
