@@ -48,12 +48,21 @@ topk_kernel(const float* __restrict__ logits, int nsplit, const float* __restric
   if (t >= T) return;
   const float* row = logits + static_cast<size_t>(t) * E;
   const size_t slice = static_cast<size_t>(T) * E;
-  // logit = the sum of the K slices' partial logits, in slice order
-  auto logit_of = [&](int e) {
-    float l = row[e];
-    for (int s = 1; s < nsplit; ++s) l += row[s * slice + e];
-    return l;
-  };
+  // logit = the sum of the K slices' partial logits, in slice order; all of
+  // this lane's loads of a slice are issued together
+  float lv[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    lv[i] = (e < E) ? row[e] : 0.0f;
+  }
+  for (int s = 1; s < nsplit; ++s) {
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) lv[i] += row[s * slice + e];
+    }
+  }
   const bool use_bias = (bias != nullptr) && (score_fn != MOE_SCORE_SOFTMAX);
 
   float key[NPL];
@@ -63,7 +72,7 @@ topk_kernel(const float* __restrict__ logits, int nsplit, const float* __restric
     const int e = lane + 32 * i;
     float kv = -INFINITY;
     if (e < E) {
-      const float l = logit_of(e);
+      const float l = lv[i];
       lmax = fmaxf(lmax, l);
       kv = (score_fn == MOE_SCORE_SOFTMAX) ? l : score_of(l, score_fn) + (use_bias ? bias[e] : 0.0f);
     }
@@ -114,7 +123,8 @@ topk_kernel(const float* __restrict__ logits, int nsplit, const float* __restric
 
   float s = 0.0f;
   if (lane < k) {
-    const float l = logit_of(my_idx);
+    float l = row[my_idx];
+    for (int s = 1; s < nsplit; ++s) l += row[s * slice + my_idx];
     s = (score_fn == MOE_SCORE_SOFTMAX) ? expf(l - lmax) : score_of(l, score_fn);
   }
   float denom;

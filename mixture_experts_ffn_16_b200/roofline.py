@@ -78,9 +78,9 @@ def block_cost(cfg, touched=None):
 # valid only while the GEMM code is the one that was captured (sha256 prefix
 # of the source without comments).
 NCU_TRAFFIC = {
-    ("prefill_softmax", "route"): (17.9e6, "103616b7ddfab397"),
-    ("prefill_softmax", "gate_up"): (1109.8e6, "103616b7ddfab397"),
-    ("prefill_softmax", "down"): (746.4e6, "103616b7ddfab397"),
+    ("prefill_softmax", "route"): (17.9e6, "5335669b4bc0657e"),
+    ("prefill_softmax", "gate_up"): (1108.3e6, "5335669b4bc0657e"),
+    ("prefill_softmax", "down"): (747.3e6, "5335669b4bc0657e"),
 }
 
 
