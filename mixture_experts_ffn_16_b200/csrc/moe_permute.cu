@@ -131,13 +131,14 @@ struct ScanArgs {
 
 __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) {
   chain_wait();
-  // Experts per thread: E <= 2048 -> at most 2.
+  // Experts per thread, contiguous: one up to E = 1024, else two.
   constexpr int kPer = (kMaxE + kScanThreads - 1) / kScanThreads;
+  const int per = a.E > kScanThreads ? kPer : 1;
   int cnt[kPer], pad[kPer], u1[kPer], u2[kPer];
   int sp = 0, s1 = 0, s2 = 0;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
-    const int e = threadIdx.x * kPer + i;
+    const int e = (i < per) ? threadIdx.x * per + i : a.E;
     int c = 0;
     if (e < a.E) {
       // Column e of the block histogram: exclusive prefix over blocks.  The
@@ -171,7 +172,7 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) 
   int o2 = a.shared_units2 + ex.z;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
-    const int e = threadIdx.x * kPer + i;
+    const int e = (i < per) ? threadIdx.x * per + i : a.E;
     if (e < a.E) {
       a.roff[e] = ro;
       // padding rows of this expert's segment

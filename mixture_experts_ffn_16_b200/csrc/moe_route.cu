@@ -124,7 +124,7 @@ topk_kernel(const float* __restrict__ logits, int nsplit, const float* __restric
   float s = 0.0f;
   if (lane < k) {
     float l = row[my_idx];
-    for (int s = 1; s < nsplit; ++s) l += row[s * slice + my_idx];
+    for (int sl = 1; sl < nsplit; ++sl) l += row[sl * slice + my_idx];
     s = (score_fn == MOE_SCORE_SOFTMAX) ? expf(l - lmax) : score_of(l, score_fn);
   }
   float denom;
