@@ -22,7 +22,13 @@
  *     diagram ("MoE router - sigma / sqrt-softplus - bias balancing");
  *   SwiGLU experts at full width: qwen3-5-vs-gemma-4 component table, Qwen3.5
  *     routed-experts cell; shared expert added to the routed sum: same table,
- *     Qwen3.5 shared-expert cell (ungated, DeepSeek-style, is what is built).
+ *     Qwen3.5 shared-expert cell (ungated, DeepSeek-style, by default; the
+ *     Qwen3.5 per-token sigmoid gate with W_shared_gate_vec).
+ *
+ * Beyond the block itself: moe_forward_prenorm (the pre-norm RMSNorm fused in
+ * front), moe_forward_fp8 (block-scaled FP8 expert weights),
+ * moe_experts_forward (routing supplied by the caller), moe_forward_host
+ * (host buffers), the step entry points, and moe_route_noalloc.
  *
  * Conventions for every entry point
  *   - Tensors are dense, row-major, in device memory unless stated otherwise,
@@ -38,7 +44,11 @@
  *     except moe_device_status synchronises the host.
  *   - The library allocates no device memory and keeps no per-call state: all
  *     scratch lives in the caller's workspace (size from moe_workspace_bytes),
- *     which must not be used by two calls that overlap on the GPU.
+ *     which must not be used by two calls that overlap on the GPU.  (The one
+ *     exception, moe_route_noalloc, uses a scratch array inside the library.)
+ *   - Kernels are launched with programmatic stream serialisation: each waits
+ *     for the previous kernel in the stream before touching memory, so stream
+ *     order is preserved while launch latency overlaps.
  *   - On an error return nothing has been enqueued and the outputs are
  *     untouched.
  *   - Kernels never trap.  Every device-side wait is bounded; a wait that runs
