@@ -208,3 +208,16 @@ def test_fp8_argument_checks(lib):
     assert lib.moe_expert_gate_up_fp8(ctypes.byref(s), P(4096), pg, None, pg, pg, P(4096), n, None) == \
         api.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_down_fp8(ctypes.byref(s), pg, None, P(4096), n, None) == api.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", list(CONFIGS))
+def test_router_logit_slices(lib, name):
+    """The logits region holds P whole [T, E] fp32 arrays, one per K slice of
+    the router GEMM: at least one, at most 16, never more than d / 64."""
+    c = CONFIGS[name]
+    s = api.shape_of(c)
+    _, nb = api.moe_workspace_region(s, "logits")
+    one = c.T * c.E * 4
+    assert nb % one == 0
+    slices = nb // one
+    assert 1 <= slices <= min(16, c.d // 64)
