@@ -46,6 +46,10 @@
  *     scratch lives in the caller's workspace (size from moe_workspace_bytes),
  *     which must not be used by two calls that overlap on the GPU.  (The one
  *     exception, moe_route_noalloc, uses a scratch array inside the library.)
+ *   - Entry points may be called from several host threads at once, each call
+ *     with its own workspace.  The only state kept across calls is per device
+ *     and filled in once under a lock: the device's properties, the kernels'
+ *     shared-memory limits and the tensor-map encoder's address.
  *   - Kernels are launched with programmatic stream serialisation: each waits
  *     for the previous kernel in the stream before touching memory, so stream
  *     order is preserved while launch latency overlaps.

@@ -23,15 +23,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  // looked up once per process (thread-safe static initialisation); first
+  // reached from device_info, after the runtime is up
+  static const EncodeTiledFn fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+      return reinterpret_cast<EncodeTiledFn>(ptr);
+    return static_cast<EncodeTiledFn>(nullptr);
+  }();
   return fn;
 }
 
@@ -478,12 +480,22 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
   return MOE_OK;
 }
 
+std::mutex& host_state_mutex() {
+  static std::mutex m;
+  return m;
+}
+
 int device_info(DeviceInfo* info) {
   static DeviceInfo cache[64];
-  static int have[64] = {0};
+  static std::atomic<int> have[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
-  if (!have[dev]) {
+  if (!have[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(host_state_mutex());
+    if (have[dev].load(std::memory_order_relaxed)) {
+      *info = cache[dev];
+      return MOE_OK;
+    }
     DeviceInfo d;
     std::memset(&d, 0, sizeof d);
     int major = 0;
@@ -493,7 +505,7 @@ int device_info(DeviceInfo* info) {
       return MOE_ERR_CUDA;
     d.ok = (major == 10 && d.max_smem_optin >= 232448 && encode_fn() != nullptr) ? 1 : 0;
     cache[dev] = d;
-    have[dev] = 1;
+    have[dev].store(1, std::memory_order_release);
   }
   *info = cache[dev];
   return MOE_OK;
@@ -860,18 +872,21 @@ constexpr size_t kNoAllocLogitBytes = size_t(16) << 20;     // fp32 logits: T * 
 static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocHeaderBytes + kNoAllocLogitBytes];
 
 char* g_route_scratch_dev[64];    // device address of g_route_scratch, per device
-int g_route_scratch_ready[64];
+std::atomic<int> g_route_scratch_ready[64];
 
 // The host-side name g_route_scratch is not a device address: look up the
 // device address once per device (with that device current) and reuse it.
 int route_scratch_address(char** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
-  if (!g_route_scratch_ready[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_route_scratch) != cudaSuccess || ptr == nullptr) return MOE_ERR_CUDA;
-    g_route_scratch_dev[dev] = static_cast<char*>(ptr);
-    g_route_scratch_ready[dev] = 1;
+  if (!g_route_scratch_ready[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(host_state_mutex());
+    if (!g_route_scratch_ready[dev].load(std::memory_order_relaxed)) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_route_scratch) != cudaSuccess || ptr == nullptr) return MOE_ERR_CUDA;
+      g_route_scratch_dev[dev] = static_cast<char*>(ptr);
+      g_route_scratch_ready[dev].store(1, std::memory_order_release);
+    }
   }
   *out = g_route_scratch_dev[dev];
   return MOE_OK;

@@ -1265,16 +1265,9 @@ size_t gemm_pair_smem_bytes(int mode, int nmax, int* stages) {
 
 template <int MODE>
 static int launch_pair_mode(const GemmParams& prm, int grid, size_t smem, cudaStream_t st) {
-  static int configured[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
-  if (configured[dev] < static_cast<int>(smem)) {
-    if (cudaFuncSetAttribute(moe_gemm_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    configured[dev] = static_cast<int>(smem);
-  }
+  static std::atomic<int> limit[64];
+  const int rc = raise_smem_limit(moe_gemm_pair_kernel<MODE>, limit, static_cast<int>(smem));
+  if (rc != MOE_OK) return rc;
   return launch_chained(moe_gemm_pair_kernel<MODE>, dim3(grid), dim3(threads_of(MODE)), smem, st, prm) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
@@ -1312,16 +1305,9 @@ size_t gemm_f8_smem_bytes(int mode, int nmax, int* stages, int* tok_stages, int*
 
 template <int MODE, bool F8>
 static int launch_mode(const GemmParams& prm, int grid, size_t smem, cudaStream_t st) {
-  static int configured[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
-  if (configured[dev] < static_cast<int>(smem)) {
-    if (cudaFuncSetAttribute(moe_gemm_kernel<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    configured[dev] = static_cast<int>(smem);
-  }
+  static std::atomic<int> limit[64];
+  const int rc = raise_smem_limit(moe_gemm_kernel<MODE, F8>, limit, static_cast<int>(smem));
+  if (rc != MOE_OK) return rc;
   return launch_chained(moe_gemm_kernel<MODE, F8>, dim3(grid), dim3(threads_of(MODE, F8)), smem, st, prm) ==
                  cudaSuccess
              ? MOE_OK

@@ -3,8 +3,10 @@
 // libmoe.so only.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -21,6 +23,28 @@ constexpr int kTileK = 64;         // bf16 elements per 128-byte swizzled row
 constexpr int kRowPad = 16;        // expert segments are padded to this many rows (MMA N step)
 constexpr int kPermBlock = 256;    // tokens per block in the permute kernels
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
+
+// Host-side state kept per device for the life of the process (kernel
+// attributes, device queries, the no-alloc scratch address) is filled in
+// under this lock, so the entry points may be called from several host
+// threads at once.
+std::mutex& host_state_mutex();
+
+// Raises `kernel`'s dynamic shared-memory limit on the current device to at
+// least `bytes`; `limit` records per device what is set already.  The limit
+// only grows, so a launch that needs less is never refused.
+template <typename... KArgs>
+inline int raise_smem_limit(void (*kernel)(KArgs...), std::atomic<int> (&limit)[64], int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  if (limit[dev].load(std::memory_order_acquire) >= bytes) return MOE_OK;
+  std::lock_guard<std::mutex> lock(host_state_mutex());
+  if (limit[dev].load(std::memory_order_relaxed) >= bytes) return MOE_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  limit[dev].store(bytes, std::memory_order_release);
+  return MOE_OK;
+}
 
 #ifdef __CUDACC__
 // Every kernel of the block is launched with programmatic stream

@@ -254,15 +254,13 @@ int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, 
   int32_t* blkcnt = reinterpret_cast<int32_t*>(ws + p.blkcnt);
   uint32_t* err = reinterpret_cast<uint32_t*>(ws + p.err);
   const size_t msmem = static_cast<size_t>(kWarps) * p.E * sizeof(uint32_t);
-  static int configured[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
-  if (!configured[dev]) {
+  {
+    // set once per device to the largest E's mask array
+    static std::atomic<int> count_limit[64], scatter_limit[64];
     const int mx = kWarps * kMaxE * static_cast<int>(sizeof(uint32_t));
-    if (cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess ||
-        cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    configured[dev] = 1;
+    int rc = raise_smem_limit(permute_count_kernel, count_limit, mx);
+    if (rc == MOE_OK) rc = raise_smem_limit(permute_scatter_kernel, scatter_limit, mx);
+    if (rc != MOE_OK) return rc;
   }
   if (launch_chained(permute_count_kernel, dim3(p.nb), dim3(kPermBlock), msmem, st, topk_idx, p.T, p.E, p.k, blkcnt,
                      err) != cudaSuccess)
