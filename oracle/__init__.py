@@ -30,12 +30,18 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 SOFTMAX, SIGMOID, SQRT_SOFTPLUS = 0, 1, 2
 SCORE_FNS = {"softmax": SOFTMAX, "sigmoid": SIGMOID, "sqrt_softplus": SQRT_SOFTPLUS}
 
+# A prebuilt library loaded instead of liboracle.so.  Only the planted-mistake
+# tests set it, to run the pins against mutated copies of moe_oracle.c.
+_OVERRIDE = os.environ.get("MOE_ORACLE_LIB") or None
+
 _lock = threading.Lock()
 _lib = None
 
 
 def build(force: bool = False) -> str:
     """Compile moe_oracle.c into liboracle.so (gcc, -O2, no fast-math)."""
+    if _OVERRIDE:
+        return _OVERRIDE
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
@@ -48,8 +54,7 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB)
+            lib = ctypes.CDLL(build())
             P = ctypes.c_void_p
             i = ctypes.c_int
             lib.oracle_moe_forward.restype = i
