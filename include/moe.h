@@ -37,8 +37,9 @@
  *        x [T,d]  W_router [E,d]  W_gate, W_up [E,f,d]  W_down [E,d,f]
  *        W_shared_gate, W_shared_up [S,fs,d]  W_shared_down [S,d,fs]
  *   - Every device pointer must be 16-byte aligned; d, f and fs must be
- *     multiples of 64; 1 <= k <= min(E, 32); 1 <= E <= 2048; 0 <= S <= 8;
- *     T >= 1.  Violations return an error code and enqueue nothing.
+ *     multiples of 64 and at most 65536; 1 <= k <= min(E, 32);
+ *     1 <= E <= 2048; 0 <= S <= 8; 1 <= T <= 4,194,304.  Violations return
+ *     an error code and enqueue nothing.
  *   - `stream` is a cudaStream_t passed as a plain pointer (NULL = legacy
  *     default stream).  Work is enqueued asynchronously on it; no entry point
  *     except moe_device_status synchronises the host.

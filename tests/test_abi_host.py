@@ -70,6 +70,9 @@ def test_workspace_sizes_of_workloads(lib, name):
     (dict(d_model=100), api.MOE_ERR_UNSUPPORTED), (dict(d_ff=96), api.MOE_ERR_UNSUPPORTED),
     (dict(n_shared=1, d_ff_shared=80), api.MOE_ERR_UNSUPPORTED), (dict(E=4096), api.MOE_ERR_UNSUPPORTED),
     (dict(k=33, E=64), api.MOE_ERR_UNSUPPORTED), (dict(n_shared=9, d_ff_shared=64), api.MOE_ERR_UNSUPPORTED),
+    (dict(T=(1 << 22) + 1), api.MOE_ERR_UNSUPPORTED), (dict(d_model=65536 + 64), api.MOE_ERR_UNSUPPORTED),
+    (dict(d_ff=65536 + 64), api.MOE_ERR_UNSUPPORTED), (dict(d_ff_shared=65536 + 64), api.MOE_ERR_UNSUPPORTED),
+    (dict(n_shared=-1), api.MOE_ERR_INVALID_ARG), (dict(n_shared=1, d_ff_shared=0), api.MOE_ERR_INVALID_ARG),
 ])
 def test_invalid_shapes(lib, bad, code):
     base = dict(T=16, d_model=128, E=8, k=2, d_ff=128, n_shared=1, d_ff_shared=128)
@@ -79,6 +82,12 @@ def test_invalid_shapes(lib, bad, code):
     st = lib.moe_forward(ctypes.byref(s), *([ctypes.c_void_p(256)] * 9), None, 0, 1, 1.0,
                          *([ctypes.c_void_p(256)] * 4), 1 << 30, None)
     assert st == code
+
+
+def test_largest_supported_shape_plans(lib):
+    """The limits themselves are accepted: T = 2^22, d = f = fs = 65536."""
+    s = api.make_shape(1 << 22, 65536, 8, 2, 65536, 1, 65536)
+    assert api.moe_workspace_bytes(s) > 0
 
 
 def test_argument_checks_before_any_device_work(lib):
