@@ -20,7 +20,6 @@ import dataclasses
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time

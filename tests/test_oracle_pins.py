@@ -6,7 +6,6 @@ special case reduces to (numpy matmul, scipy expit / logaddexp), identities and
 invariants.  Together they are chosen so that a dropped term, a wrong sign or
 index, or a transposed operand anywhere in the oracle fails at least one.
 """
-import itertools
 import json
 import math
 import os
