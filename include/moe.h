@@ -1,9 +1,10 @@
 /*
  * moe.h - C ABI of libmoe.so, a B200 (sm_100a) mixture-of-experts FFN block.
  *
- * The block (archdiff.com architecture-comparison pages; blueprint diagram
- * "RMSNorm pre-norm -> router -> routed experts top-6-22 of 256-896, SwiGLU ->
- * shared expert 1-2, always active -> residual add", qwen3-5-vs-deepseek-v4):
+ * The block (archdiff.com architecture-comparison pages; in the blueprint
+ * diagram of qwen3-5-vs-deepseek-v4 a pre-norm RMSNorm feeds the router, which
+ * picks the top 6 to 22 of 256 to 896 SwiGLU experts, one or two shared
+ * experts run for every token, and a residual add follows):
  *
  *   logits   l = x W_router^T                                   (linear router)
  *   scores   s = softmax(l) | sigmoid(l) | sqrt(softplus(l))
@@ -15,11 +16,13 @@
  *            SwiGLU(x) = W_down (SiLU(W_gate x) * (W_up x)), no residual.
  *
  * Sources on the pages:
- *   softmax router "softmax, keep the top k, renormalize, no selection bias":
- *     qwen3-5-vs-deepseek-v4 component table, Qwen3.5 router cell;
- *   sqrt-softplus router with selection-only bias, "normalized and scaled by
- *     2.5": same table, DeepSeek-V4-Pro router cell; sigma form: DeepSeek-V4-Pro
- *     diagram ("MoE router - sigma / sqrt-softplus - bias balancing");
+ *   softmax router (softmax over all experts, the k largest kept and
+ *     renormalised, no bias in the choice): qwen3-5-vs-deepseek-v4 component
+ *     table, Qwen3.5 router cell;
+ *   sqrt-softplus router with a bias that only picks experts, the picked
+ *     scores renormalised and multiplied by 2.5: same table, DeepSeek-V4-Pro
+ *     router cell; sigmoid form: the router node of the DeepSeek-V4-Pro
+ *     diagram;
  *   SwiGLU experts at full width: qwen3-5-vs-gemma-4 component table, Qwen3.5
  *     routed-experts cell; shared expert added to the routed sum: same table,
  *     Qwen3.5 shared-expert cell (ungated, DeepSeek-style, by default; the
@@ -150,10 +153,10 @@ MOE_API int moe_forward_host(const moe_shape *shape,
                      void *out_host, int32_t *topk_idx_host, float *topk_w_host,
                      void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
-/* The block with its pre-norm RMSNorm fused in front (the Qwen3.5 block puts
- * "RMSNorm - pre-norm" directly before the router: qwen3-5-vs-deepseek-v4,
- * Qwen3.5 diagram; the gains are zero-centred: same page, component table,
- * Qwen3.5 residual-stream cell).
+/* The block with its pre-norm RMSNorm fused in front (the Qwen3.5 diagram of
+ * qwen3-5-vs-deepseek-v4 draws a pre-norm RMSNorm right before the router;
+ * the gains are zero-centred: same page, component table, Qwen3.5
+ * residual-stream cell).
  *   x         [T,d] bf16: the residual stream (not normalised).
  *   norm_gain [d] bf16: zero-centred gains g; the scale applied is 1 + g.
  *   norm_eps  finite, >= 0 (the pages give no value; Qwen-family models use
@@ -181,16 +184,16 @@ MOE_API int moe_rmsnorm(const moe_shape *shape, const void *x, const void *norm_
                 void *x_norm, moe_stream_t stream);
 
 /* ---- Block-scaled FP8 expert weights ----
- * The pages name an official FP8 weight release and "block-scaled FP8"
- * (qwen3-5-vs-gemma-4, component table, Qwen3.5 routed-experts cell;
- * qwen3-5-vs-deepseek-v4, blueprint diagram) but give no block size or scale
- * format.  Reading: OCP MX-style blocks of 32 consecutive elements along the
+ * The pages mention an FP8 release of the Qwen3.5 weights and block-scaled
+ * FP8 in the training blueprint (qwen3-5-vs-gemma-4, component table, Qwen3.5
+ * routed-experts cell; qwen3-5-vs-deepseek-v4, blueprint diagram) but give no
+ * block size or scale format.  Reading: OCP MX-style blocks of 32 consecutive elements along the
  * input dimension K, one power-of-two scale per block stored as its biased
  * exponent byte (UE8M0).  Element [g, r, c] of the weight is
  *     e4m3(codes[g, r, c]) * 2^(scales[g, c / 32, r] - 127)
  * with codes in the [out, in] layout of the bf16 weight and the scales
  * block-major.  E4M3 is the OCP "E4M3FN" encoding (no infinities, 0x7F/0xFF
- * NaN).  The library widens each tile to bf16 in shared memory; the widened
+ * NaN).  The library widens each tile to bf16 in tensor memory; the widened
  * value is exact whenever it is representable in bf16 (scale bytes 10..246
  * for finite codes), so the block then computes exactly what moe_forward
  * computes on the widened weights, while HBM moves half the weight bytes. */

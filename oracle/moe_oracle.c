@@ -10,17 +10,19 @@
  *
  * Source of the method (archdiff.com architecture-comparison pages on
  * Qwen3.5-397B-A17B, DeepSeek-V4-Pro, Qwen3.8, Gemma 4 and DeepSeek-V4.1-Flash):
- *   - "Softmax top-k router": a linear router scores the experts; softmax,
- *     keep the top k, renormalise; no selection bias.
+ *   - Qwen3.5's router: a linear map gives one score per expert, a softmax
+ *     turns them into probabilities, the k largest are kept and renormalised,
+ *     and no bias takes part in the choice.
  *     (qwen3-5-vs-deepseek-v4, component table, Qwen3.5 router cell;
  *      qwen3-5-vs-gemma-4, component table, Qwen3.5 router cell)
- *   - "MoE router - sigma / sqrt-softplus - bias balancing": sqrt(softplus)
- *     affinities with a per-expert bias used only to pick the top k; the
- *     selected scores are normalised and scaled.
+ *   - DeepSeek-V4-Pro's router: sqrt(softplus) affinities; a per-expert bias
+ *     is added only while the k experts are chosen; the chosen affinities are
+ *     renormalised and multiplied by a constant.  The router node of its
+ *     diagram names the sigmoid form beside it.
  *     (qwen3-5-vs-deepseek-v4, DeepSeek-V4-Pro diagram and router cell)
- *   - "Routed experts - top-6-22 of 256-896 - SwiGLU" and
- *     "Shared expert - 1-2 - always active", then the residual add as a
- *     separate node (qwen3-5-vs-deepseek-v4, Qwen3.5 diagram).
+ *   - The routed SwiGLU experts (the top 6 to 22 of 256 to 896) and one or
+ *     two shared experts that every token uses; the residual add is drawn as
+ *     its own node after the block (qwen3-5-vs-deepseek-v4, Qwen3.5 diagram).
  *   - SwiGLU experts at full model width, no latent projection
  *     (qwen3-5-vs-gemma-4, component table, Qwen3.5 routed-experts cell).
  *   - The shared expert's output is added to the routed sum
@@ -332,7 +334,7 @@ int oracle_moe_forward(int T, int d, int E, int k, int f, int S, int fs,
 
 /* ------------------------------------------------------------------ RMSNorm
  * The pre-norm RMSNorm that produces the block's input (qwen3-5-vs-deepseek-v4,
- * Qwen3.5 diagram: "RMSNorm - pre-norm" directly before the router), with
+ * Qwen3.5 diagram: the pre-norm RMSNorm node right before the router), with
  * zero-centred gains (same page, component table, Qwen3.5 residual-stream
  * cell): the stored gain g is centred on zero, so the scale applied is 1 + g.
  *
@@ -388,9 +390,10 @@ int oracle_rmsnorm(int T, int d, const uint16_t *x, const uint16_t *gain, double
 }
 
 /* ------------------------------------------------------------------ FP8 weights
- * Block-scaled FP8 expert weights (the pages name an official FP8 weight
- * release and "block-scaled FP8": qwen3-5-vs-gemma-4, component table,
- * Qwen3.5 routed-experts cell; qwen3-5-vs-deepseek-v4, blueprint diagram).
+ * Block-scaled FP8 expert weights (the pages mention an FP8 release of the
+ * Qwen3.5 weights and block-scaled FP8 in the training blueprint:
+ * qwen3-5-vs-gemma-4, component table, Qwen3.5 routed-experts cell;
+ * qwen3-5-vs-deepseek-v4, blueprint diagram).
  * The pages give no block size or scale format.  Reading: OCP MX-style
  * blocks of 32 consecutive elements along the input dimension K, each with
  * one power-of-two scale stored as an unbiased-exponent byte (UE8M0):

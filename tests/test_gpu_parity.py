@@ -135,8 +135,8 @@ GATED = [
 
 @pytest.mark.parametrize("cfg", GATED, ids=lambda c: c.name)
 def test_gated_shared_expert_every_token(oracle_mod, cfg):
-    """The Qwen3.5 shared expert: scaled per token by sigmoid(w . x) before it
-    is added to the routed sum."""
+    """The Qwen3.5 shared expert: its output is scaled per token by
+    sigmoid(w . x), then joins the sum over the routed experts."""
     rep, _ = parity_case(oracle_mod, cfg)
     assert rep["tokens"] == cfg.T
 

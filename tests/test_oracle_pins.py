@@ -500,9 +500,9 @@ def test_rmsnorm_eps_closed_form_and_zero_row(oracle_mod):
 
 
 # ---------------------------------------------------------------- block-scaled FP8 weights
-# w = e4m3(q) * 2^(s - 127), one UE8M0 scale per 32 elements along K (reading of
-# "block-scaled FP8": qwen3-5-vs-deepseek-v4 blueprint diagram; qwen3-5-vs-gemma-4,
-# Qwen3.5 routed-experts cell).
+# w = e4m3(q) * 2^(s - 127), one UE8M0 scale per 32 elements along K (the reading
+# taken of block-scaled FP8: qwen3-5-vs-deepseek-v4 blueprint diagram;
+# qwen3-5-vs-gemma-4, Qwen3.5 routed-experts cell).
 
 @pytest.mark.parametrize("code,value", [
     (0x38, 1.0), (0xB8, -1.0), (0x7E, 448.0), (0xFE, -448.0), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9),
