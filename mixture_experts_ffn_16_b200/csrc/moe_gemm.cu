@@ -6,7 +6,10 @@
 //
 // One persistent, warp-specialised kernel template serves all three.  A work
 // unit is (group g, 128-row block of the weight matrix, a run of n <= nmax
-// consecutive rows of the group's row segment).  The GEMM is "swap-AB": the
+// consecutive rows of the group's row segment); for the router, g is a slice
+// of d instead when the plan splits K, each slice writing its own partial
+// logits.  A CTA-pair form (cta_group::2, moe_gemm_pair_kernel) serves the
+// gate/up GEMM of large experts.  The GEMM is "swap-AB": the
 // 128 weight rows are the MMA's M side and the unit's tokens its N side
 // (n a multiple of 16), so an expert with few tokens costs n/16 MMA columns,
 // not a padded 128-row tile.
