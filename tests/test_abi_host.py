@@ -230,3 +230,29 @@ def test_router_logit_slices(lib, name):
     assert nb % one == 0
     slices = nb // one
     assert 1 <= slices <= min(16, c.d // 64)
+
+
+def test_binding_marshalling_checks():
+    """The Python binding checks device, dtype, shape and layout before it
+    hands a pointer to the library."""
+    import torch
+    bf = torch.bfloat16
+    t = torch.zeros(4, 8, dtype=bf)
+    assert api._p(None) is None
+    assert api._p(256).value == 256
+    with pytest.raises(TypeError):
+        api._p([1, 2], bf, (4, 8), "x")
+    with pytest.raises(ValueError, match="CUDA"):
+        api._p(t, bf, (4, 8), "x")                      # a host tensor where device memory is expected
+    assert api._p(t, bf, (4, 8), "x", host=True).value == t.data_ptr()
+    with pytest.raises(TypeError, match="bfloat16"):
+        api._p(t.float(), bf, (4, 8), "x", host=True)
+    with pytest.raises(ValueError, match="shape"):
+        api._p(t, bf, (8, 4), "x", host=True)
+    with pytest.raises(ValueError, match="contiguous"):
+        api._p(t.t(), bf, (8, 4), "x", host=True)
+    s = api.make_shape(4, 8, 2, 1, 64, 0, 0)
+    with pytest.raises(ValueError, match="CUDA"):
+        api.moe_forward(s, t, torch.zeros(2, 8, dtype=bf), None, None, None, None, None, None, None,
+                        "softmax", True, 1.0, torch.zeros(4, 8, dtype=bf), torch.zeros(4, 1, dtype=torch.int32),
+                        torch.zeros(4, 1), None, stream=0)
