@@ -293,16 +293,18 @@ MOE_API int moe_experts_forward(const moe_shape *shape, const void *x, const int
 /* Introspection of the workspace layout, for tests and debugging.  Regions:
  *   MOE_WS_LOGITS   fp32 [P,T,E] router logits (after moe_route) as P partial
  *                                sums over slices of d, added in slice order
- *                                (P = 1 unless the batch is too small to
- *                                fill the GPU with token runs alone)
+ *                                (P > 1 when the plan splits d: to fill the
+ *                                SMs with small batches, or where two slices
+ *                                load fewer bytes per SM; P <= 16)
  *   MOE_WS_COUNTS   int32 [E]    tokens per expert (after moe_permute)
  *   MOE_WS_OFFSETS  int32 [E+1]  first row of each expert's segment; segments
- *                                are padded to 16 rows; [E] = total rows
+ *                                are padded to p rows (p = 16, or 32 when
+ *                                experts average 256+ rows); [E] = total rows
  *   MOE_WS_PERM     int32 [rows] token of each routed row (padding rows: 0)
  *   MOE_WS_ROW_W    fp32 [rows]  combine weight of each routed row (padding: 0)
  *   MOE_WS_INV      int32 [T,k]  row of each (token, slot)
  *   MOE_WS_H        bf16 [rows,f]   routed hidden rows (after moe_expert_gate_up)
- *   MOE_WS_H_SHARED bf16 [S,Tp,fs]  shared hidden rows, Tp = T rounded up to 16
+ *   MOE_WS_H_SHARED bf16 [S,Tp,fs]  shared hidden rows, Tp = T rounded up to p
  *   MOE_WS_Y        bf16 [rows,d]   weighted routed outputs (after moe_expert_down)
  *   MOE_WS_Y_SHARED bf16 [S,Tp,d]   shared outputs
  *   MOE_WS_X_STAGE  bf16 [T,d]      token rows the library staged: x copied
