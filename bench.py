@@ -5,10 +5,17 @@
 
 A step is one pass of the whole block (router GEMM, top-k, permute, gate/up
 GEMM, down GEMM, combine) over one batch of T tokens whose inputs are already
-in HBM.  Default workload: prefill with a softmax top-8 router (T=4096,
-d=2048, E=256, d_ff=512, one shared expert of 512), seeded synthetic inputs.
+in HBM.  Default workload: the large load-imbalanced layer (T=16384,
+d=7168, E=896 routed experts, top-22 softmax router with Zipf-rank skew,
+d_ff=512, two shared experts of 1024), seeded synthetic inputs.  The same
+run also times the other full-size workloads (prefill softmax, prefill
+sigmoid, decode sqrt-softplus) and reports them under "workloads".
 With N GPUs (torchrun) every rank runs its own replica on its own batch
 (weak scaling, no collective on the data path); the time is the max over ranks.
+
+The CPU-baseline leg times the fp64 oracle on a seeded token sample of the
+timed workload and compares the GPU's results for those tokens with it
+("parity": tokens checked, near-tie tokens, order swaps, error ratios).
 
 --impl reference times the fp64 CPU oracle (the slow plain definition) on a
 bounded sample of the same workload on rank 0; other ranks exit at once.
@@ -39,6 +46,7 @@ from mixture_experts_ffn_16_b200.roofline import (block_cost, kernel_costs, meas
 METRIC = "MoE-layer tokens/sec at 1 B200; % bf16 tensor peak (prefill) / % HBM BW (decode)"
 STAGES = ["route", "permute", "gate_up", "down", "combine"]
 LAUNCHES_PER_STEP = {"route": 2, "permute": 3, "gate_up": 1, "down": 1, "combine": 1}
+EXTRA_WORKLOADS = ["prefill_softmax", "prefill_sigmoid", "decode_sqrt_softplus", "large_imbalanced"]
 REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
@@ -48,25 +56,49 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="prefill_softmax", choices=list(CONFIGS))
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="large_imbalanced", choices=list(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip timing the other workloads")
+    ap.add_argument("--extra-steps", type=int, default=100, help="timed steps of each other workload (min K)")
     ap.add_argument("--variant", default="", choices=["", "gated_shared", "external_routing", "prenorm", "fp8"],
                     help="gated_shared: Qwen3.5-style sigmoid gate on the shared experts; "
                          "external_routing: routing supplied by the caller (steps a3..a7 only); "
-                         "prenorm: the pre-norm RMSNorm (zero-centred gains) fused in front; "
+                         "prenorm: the pre-norm RMSNorm (zero-centred gains) in front; "
                          "fp8: block-scaled FP8 expert weights")
     return ap.parse_args()
+
+
+def config_dict(cfg, variant, n_gpus):
+    """The workload as both arms report it (the same dict on both)."""
+    return {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "E": cfg.E, "k": cfg.k, "d_ff": cfg.f,
+            "n_shared": cfg.S, "d_ff_shared": cfg.fs, "score_fn": cfg.score_fn, "norm_topk": cfg.norm_topk,
+            "route_scale": cfg.route_scale, "expert_bias_std": cfg.bias_std, "skew": cfg.skew or "none",
+            "variant": variant or "base",
+            "expert_weights": "fp8 e4m3 + ue8m0 scale per 32" if cfg.fp8 else "bf16",
+            "l2": "no flush: inputs larger than L2 (expert weights %.2f GB per step)" % (
+                weight_bytes(cfg) * (cfg.E * 3 * cfg.f * cfg.d + cfg.S * 3 * cfg.fs * cfg.d) / 1e9),
+            "parallelism": "replicas" if n_gpus > 1 else "single GPU"}
+
+
+def variant_cfg(cfg, variant):
+    if variant == "gated_shared":
+        return dataclasses.replace(cfg, shared_gate=True)
+    if variant == "prenorm":
+        return dataclasses.replace(cfg, prenorm=True)
+    if variant == "fp8":
+        return dataclasses.replace(cfg, fp8=True)
+    return cfg
 
 
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML while running."""
 
-    def __init__(self, device_index, period_s=0.01):
+    def __init__(self, device_index, period_s=0.005):
         self.samples = []
         self.max_mhz = None
         self.period = period_s
@@ -114,7 +146,7 @@ class ClockSampler:
             bits |= s[1]
         reasons = [name for b, name in REASON_BITS.items() if bits & b]
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(self.samples)}
+                "samples": len(self.samples), "period_ms": 1e3 * self.period}
 
 
 def dist_setup(n_gpus):
@@ -154,25 +186,58 @@ def barrier(world):
         dist.barrier()
 
 
-def cpu_oracle_rate(cfg, host, target_s, seed=12345):
-    """Time the oracle on a seeded token sample sized to about target_s seconds."""
+# ---------------------------------------------------------------- the oracle legs (CPU)
+
+def oracle_host_args(oracle, cfg, inp):
+    """Host inputs of the oracle for this workload: the drawn tensors, with the
+    FP8 expert weights replaced by the oracle's own dequantisation and, for the
+    pre-norm variant, x by the oracle's RMSNorm of it."""
+    from mixture_experts_ffn_16_b200.inputs import bf16_bits
+    host = oracle_args(inp)
+    if cfg.fp8:
+        for name in ("W_gate", "W_up", "W_down", "W_shared_gate", "W_shared_up", "W_shared_down"):
+            f8 = inp.get(name + "_f8")
+            if f8 is not None:
+                host[name] = oracle.dequant_mxfp8(f8[0].cpu().numpy(), f8[1].cpu().numpy())
+    if cfg.prenorm:
+        host["x"] = oracle.rmsnorm(host["x"], bf16_bits(inp["norm_gain"]), float(np.float32(cfg.norm_eps)))["y_bits"]
+    return host
+
+
+def cpu_baseline_leg(cfg, inp, gpu_result, target_s, seed=12345):
+    """Time the oracle on a seeded token sample sized to about target_s seconds
+    of host CPU work, then compare the GPU's results for those tokens with the
+    oracle's (index, near-tie, weight and output rules of the parity tests)."""
     import oracle
+    from oracle.parity import check_parity
     oracle.build()
+    host = oracle_host_args(oracle, cfg, inp)
     threads = os.cpu_count() or 1
+    kw = dict(k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk, route_scale=cfg.route_scale,
+              n_threads=threads)
     rng = np.random.default_rng(seed)
     n = min(cfg.T, max(threads, 8))
     t0 = time.perf_counter()
-    oracle.forward(**host, k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk,
-                   route_scale=cfg.route_scale, tokens=rng.choice(cfg.T, n, replace=False).astype(np.int32),
-                   n_threads=threads)
+    oracle.forward(**host, tokens=np.sort(rng.choice(cfg.T, n, replace=False)).astype(np.int32), **kw)
     dt = time.perf_counter() - t0
     n2 = int(min(cfg.T, max(n, n * target_s / max(dt, 1e-6))))
-    toks = rng.choice(cfg.T, n2, replace=False).astype(np.int32)
+    toks = np.sort(rng.choice(cfg.T, n2, replace=False)).astype(np.int32)
     t0 = time.perf_counter()
-    oracle.forward(**host, k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk,
-                   route_scale=cfg.route_scale, tokens=toks, n_threads=threads)
+    ref = oracle.forward(**host, tokens=toks, want_logits=True, **kw)
     dt = time.perf_counter() - t0
-    return n2 / dt, threads, n2, dt
+    cpu = {"value": n2 / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "sample": f"{n2} seeded tokens of {cfg.name} (full block per token, fp64), {dt:.1f} s"}
+    out, idx, w = gpu_result
+    try:
+        rep = check_parity(oracle, cfg, host, out[toks], idx[toks], w[toks], tokens=toks, ref=ref,
+                           n_threads=threads)
+        parity = {"ok": True, "tokens_checked": rep["tokens"], "boundary_ties": rep["boundary_ties"],
+                  "order_swaps": rep["order_swaps"], "max_err_ratio": rep["err_ratio"],
+                  "max_w_rel": rep["max_w_rel"], "tolerance": "max|err| <= 2e-2 max|oracle|; weights rtol 1e-5",
+                  "sample": "the cpu_baseline tokens"}
+    except AssertionError as e:
+        parity = {"ok": False, "tokens_checked": n2, "error": str(e)[:400]}
+    return cpu, parity
 
 
 def run_reference(args, cfg):
@@ -184,16 +249,16 @@ def run_reference(args, cfg):
     oracle.build()
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_inputs(cfg, device=dev)
-    host = oracle_args(inp)
+    host = oracle_host_args(oracle, cfg, inp)
     del inp
     threads = os.cpu_count() or 1
+    kw = dict(k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk, route_scale=cfg.route_scale,
+              n_threads=threads)
     rng = np.random.default_rng(777)
     # calibrate, then size each step so that warmup + steps take about 120 s
     n0 = min(cfg.T, max(threads, 4))
     t0 = time.perf_counter()
-    oracle.forward(**host, k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk,
-                   route_scale=cfg.route_scale, tokens=rng.choice(cfg.T, n0, replace=False).astype(np.int32),
-                   n_threads=threads)
+    oracle.forward(**host, tokens=rng.choice(cfg.T, n0, replace=False).astype(np.int32), **kw)
     rate = n0 / (time.perf_counter() - t0)
     per_step_s = 120.0 / max(1, args.steps + args.warmup)
     n = int(max(1, min(cfg.T, rate * per_step_s)))
@@ -201,8 +266,7 @@ def run_reference(args, cfg):
     for i in range(args.warmup + args.steps):
         toks = rng.choice(cfg.T, n, replace=False).astype(np.int32)
         t0 = time.perf_counter()
-        oracle.forward(**host, k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk,
-                       route_scale=cfg.route_scale, tokens=toks, n_threads=threads)
+        oracle.forward(**host, tokens=toks, **kw)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             total_tok += n
@@ -212,9 +276,7 @@ def run_reference(args, cfg):
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference",
-            "config": {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "E": cfg.E, "k": cfg.k,
-                       "d_ff": cfg.f, "n_shared": cfg.S, "d_ff_shared": cfg.fs, "score_fn": cfg.score_fn},
+            "impl": "reference", "config": config_dict(cfg, args.variant, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -222,40 +284,45 @@ def run_reference(args, cfg):
     return 0
 
 
-def run_ours(args, cfg):
-    world, rank, local = dist_setup(args.gpus)
-    api.load()
-    dev = torch.device("cuda", local if world > 1 else 0)
-    inp = make_inputs(cfg, device=dev, seed=replica_seed(cfg, rank))
-    layer = api.MoELayer(cfg, inp, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    s = layer.shape
+# ---------------------------------------------------------------- the CUDA path
 
-    external = args.variant == "external_routing"
-    if external:
-        # the caller's routing: computed once, outside the timed steps
-        ext_idx, ext_w = layer.topk_idx.clone(), layer.topk_w.clone()
-        api.moe_route(s, inp["x"], inp["W_router"], inp["expert_bias"], cfg.score_fn, cfg.norm_topk,
-                      cfg.route_scale, ext_idx, ext_w, layer.workspace, stream)
+class Runner:
+    """One workload's inputs, workspace and step (all through the C ABI)."""
 
-    xb = inp["x"]                       # the rows the block reads
-    if cfg.prenorm:
-        xb = api.workspace_view(layer.workspace, s, "x_stage", torch.bfloat16, (cfg.T, cfg.d))
+    def __init__(self, cfg, variant, dev, seed):
+        self.cfg, self.variant, self.dev = cfg, variant, dev
+        self.inp = make_inputs(cfg, device=dev, seed=seed)
+        self.layer = api.MoELayer(cfg, self.inp, device=dev)
+        self.stream = torch.cuda.current_stream(dev)
+        self.external = variant == "external_routing"
+        s, inp, layer = self.layer.shape, self.inp, self.layer
+        if self.external:
+            # the caller's routing: computed once, outside the timed steps
+            self.ext_idx, self.ext_w = layer.topk_idx.clone(), layer.topk_w.clone()
+            api.moe_route(s, inp["x"], inp["W_router"], inp["expert_bias"], cfg.score_fn, cfg.norm_topk,
+                          cfg.route_scale, self.ext_idx, self.ext_w, layer.workspace, self.stream)
+        self.xb = inp["x"]                       # the rows the block reads
+        if cfg.prenorm:
+            self.xb = api.workspace_view(layer.workspace, s, "x_stage", torch.bfloat16, (cfg.T, cfg.d))
 
-    def step(ev=None):
-        t, c = inp, cfg
+    def launches_per_step(self):
+        return (sum(LAUNCHES_PER_STEP.values()) - (LAUNCHES_PER_STEP["route"] if self.external else 0)
+                + (1 if self.cfg.prenorm else 0))
+
+    def step(self, ev=None):
+        t, c, s, layer, stream, xb = self.inp, self.cfg, self.layer.shape, self.layer, self.stream, self.xb
         if ev is not None:
             ev[0].record(stream)
-        if cfg.prenorm:
+        if c.prenorm:
             api.moe_rmsnorm(s, t["x"], t["norm_gain"], c.norm_eps, xb, stream)
-        if not external:
+        if not self.external:
             api.moe_route(s, xb, t["W_router"], t["expert_bias"], c.score_fn, c.norm_topk, c.route_scale,
                           layer.topk_idx, layer.topk_w, layer.workspace, stream)
         if ev is not None:
             ev[1].record(stream)
         (api.moe_permute_fp8 if c.fp8 else api.moe_permute)(
-            s, ext_idx if external else layer.topk_idx, ext_w if external else layer.topk_w, layer.workspace,
-            stream)
+            s, self.ext_idx if self.external else layer.topk_idx, self.ext_w if self.external else layer.topk_w,
+            layer.workspace, stream)
         if ev is not None:
             ev[2].record(stream)
         if c.fp8:
@@ -272,152 +339,205 @@ def run_ours(args, cfg):
             api.moe_expert_down(s, t["W_down"], t["W_shared_down"], layer.workspace, stream)
         if ev is not None:
             ev[4].record(stream)
-        api.moe_combine(s, layer.out, layer.workspace, stream, x=xb,
-                        W_shared_gate_vec=t.get("W_shared_gate_vec"))
+        api.moe_combine(s, layer.out, layer.workspace, stream, x=xb, W_shared_gate_vec=t.get("W_shared_gate_vec"))
         if ev is not None:
             ev[5].record(stream)
 
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize()
-    st = api.moe_device_status(layer.workspace, stream)
-    if st != api.MOE_OK:
-        raise RuntimeError(f"device status after warm-up: {api.status_string(st)}")
-    idx_host = (ext_idx if external else layer.topk_idx).cpu().numpy()
-    load = np.bincount(idx_host.ravel(), minlength=cfg.E)
-    touched = int((load > 0).sum())
-    expert_load = {"max": int(load.max()), "median": float(np.median(load)), "min": int(load.min()),
-                   "empty": int((load == 0).sum())}
+    def routing(self):
+        return self.ext_idx if self.external else self.layer.topk_idx
 
-    K = args.steps
+    def results_host(self):
+        """out, topk_idx, topk_w of the last step as host numpy arrays."""
+        idx = self.routing()
+        w = self.ext_w if self.external else self.layer.topk_w
+        return (self.layer.out.float().cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy())
+
+    def check_status(self, when):
+        st = api.moe_device_status(self.layer.workspace, self.stream)
+        if st != api.MOE_OK:
+            raise RuntimeError(f"{self.cfg.name}: device status {when}: {api.status_string(st)}")
+
+
+def time_steps(run, K, W, world):
+    """W untimed steps, then K steps timed with CUDA events on the launching
+    stream (events between the steps' entry points give each kernel's time),
+    bracketed by a barrier and a synchronize; clocks sampled meanwhile."""
+    for _ in range(max(3, W)):
+        run.step()
+    torch.cuda.synchronize()
+    run.check_status("after warm-up")
+    load = np.bincount(run.routing().cpu().numpy().ravel(), minlength=run.cfg.E)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clk:
+    with ClockSampler(run.dev.index) as clk:
         for i in range(K):
-            step(evs[i])
+            run.step(evs[i])
         torch.cuda.synchronize()
     barrier(world)
-    elapsed_ms = evs[0][0].elapsed_time(evs[-1][5])
+    elapsed_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][5]), world)
     stage_ms = {name: 0.0 for name in STAGES}
     for ev in evs:
         for j, name in enumerate(STAGES):
             stage_ms[name] += ev[j].elapsed_time(ev[j + 1])
-    stage_avg_us = {n: 1e3 * v / K for n, v in stage_ms.items()}
-    step_median_ms = float(np.median([ev[0].elapsed_time(ev[5]) for ev in evs]))
-    elapsed_ms = max_over_ranks(elapsed_ms, world)
-    st = api.moe_device_status(layer.workspace, stream)
-    if st != api.MOE_OK:
-        raise RuntimeError(f"device status after timing: {api.status_string(st)}")
+    run.check_status("after timing")
+    return {"elapsed_ms": elapsed_ms, "stage_avg_us": {n: 1e3 * v / K for n, v in stage_ms.items()},
+            "step_median_ms": float(np.median([ev[0].elapsed_time(ev[5]) for ev in evs])),
+            "clocks": clk.summary(), "touched": int((load > 0).sum()),
+            "expert_load": {"max": int(load.max()), "median": float(np.median(load)), "min": int(load.min()),
+                            "empty": int((load == 0).sum())}}
 
-    # End to end through the public host-buffer entry point.  Like a server
-    # that feeds successive batches, the steps rotate over three streams,
-    # each with its own workspace and page-locked buffers, so one batch's
-    # host<->device copies overlap the other batch's kernels.  Every step
-    # still copies its x in and its out / topk_idx / topk_w back inside the
-    # timed region.
-    e2e = None
-    # the host-buffer entry point runs the whole block on raw x with bf16
-    # weights: it has no caller-routing, pre-norm or FP8 form, so those
-    # variants report no e2e figure
-    if not args.no_e2e and not external and not cfg.prenorm and not cfg.fp8:
-        lanes = []
-        NL = 3
-        for li in range(NL):
-            st_l = stream if li == 0 else torch.cuda.Stream(dev)
-            lanes.append(dict(
-                stream=st_l,
-                ws=layer.workspace if li == 0 else api.alloc_workspace(s, dev),
-                xh=inp["x"].cpu().pin_memory(),
-                oh=torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16).pin_memory(),
-                ih=torch.empty((cfg.T, cfg.k), dtype=torch.int32).pin_memory(),
-                wh=torch.empty((cfg.T, cfg.k), dtype=torch.float32).pin_memory()))
 
-        def host_step(i):
-            L = lanes[i % NL]
-            api.moe_forward_host(s, L["xh"], inp["W_router"], inp["expert_bias"], inp["W_gate"], inp["W_up"],
-                                 inp["W_down"], inp["W_shared_gate"], inp["W_shared_up"], inp["W_shared_down"],
-                                 cfg.score_fn, cfg.norm_topk, cfg.route_scale, L["oh"], L["ih"], L["wh"], L["ws"],
-                                 L["stream"], W_shared_gate_vec=inp.get("W_shared_gate_vec"))
-        for i in range(max(2 * NL, args.warmup)):
-            host_step(i)
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        ends = [torch.cuda.Event(enable_timing=True) for _ in lanes]
-        barrier(world)
-        torch.cuda.synchronize()
-        e0.record(lanes[0]["stream"])
-        for L in lanes[1:]:
-            L["stream"].wait_event(e0)
-        for i in range(K):
-            host_step(i)
-        for L, ev in zip(lanes, ends):
-            ev.record(L["stream"])
-        torch.cuda.synchronize()
-        barrier(world)
-        for L in lanes:
-            st_chk = api.moe_device_status(L["ws"], L["stream"])
-            if st_chk != api.MOE_OK:
-                raise RuntimeError(f"device status after e2e: {api.status_string(st_chk)}")
-        e2e_ms = max_over_ranks(max(e0.elapsed_time(ev) for ev in ends), world)
-        e2e = {"value": world * cfg.T * K / (e2e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": cfg.T * cfg.d * 2,
-               "d2h_bytes_per_step": cfg.T * cfg.d * 2 + cfg.T * cfg.k * 8,
-               "streams": NL}
-
-    value = world * cfg.T * K / (elapsed_ms / 1e3)
+def roofline_of(cfg, tm, K, variant):
+    """The dominant kernel against its binding roof, and the whole step."""
     peaks = measured_peaks()
-    costs = kernel_costs(cfg, touched)
-    dom = max(STAGES, key=lambda n: stage_avg_us[n])
+    costs = kernel_costs(cfg, tm["touched"])
+    st = tm["stage_avg_us"]
+    dom = max(STAGES, key=lambda n: st[n])
     fl, by = costs[dom]
-    t_s = stage_avg_us[dom] * 1e-6
+    t_s = st[dom] * 1e-6
     t_mem = by / (peaks["hbm_gbs"] * 1e9)
     t_math = fl / (peaks["bf16_tflops"] * 1e12)
     if t_math > t_mem:
         roof = {"bound": "tensor", "achieved": fl / t_s / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        roof["frac_of_sustained"] = roof["achieved"] / peaks["bf16_tflops_sustained"]
     else:
         roof = {"bound": "hbm", "achieved": by / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     # the committed counters are those of the base (bf16, no prologue) kernels
-    roof["traffic"] = measured_traffic(cfg.name, dom) if not args.variant else None
-    roof["kernel"] = dom
-    roof["algorithmic_bytes"] = by
-    roof["algorithmic_flops"] = fl
-    roof["avg_launch_us"] = stage_avg_us[dom]
-    roof["peak_source"] = peaks["source"]
-    bfl, bby = block_cost(cfg, touched)
-    ms_step = elapsed_ms / K
-    step_roof = {"flops": bfl, "bytes": bby,
-                 "tensor_frac": bfl / (ms_step * 1e-3) / (peaks["bf16_tflops"] * 1e12),
-                 "hbm_frac": bby / (ms_step * 1e-3) / (peaks["hbm_gbs"] * 1e9)}
-    step_roof["binding_frac"] = max(step_roof["tensor_frac"], step_roof["hbm_frac"])
+    roof["traffic"] = measured_traffic(cfg.name, dom) if not variant else None
+    roof.update(kernel=dom, algorithmic_bytes=by, algorithmic_flops=fl, avg_launch_us=st[dom],
+                peak_source=peaks["source"] + (" burst" if roof["bound"] == "tensor" else ""))
+    bfl, bby = block_cost(cfg, tm["touched"])
+    ms_step = tm["elapsed_ms"] / K
+    step = {"flops": bfl, "bytes": bby,
+            "tensor_frac": bfl / (ms_step * 1e-3) / (peaks["bf16_tflops"] * 1e12),
+            "hbm_frac": bby / (ms_step * 1e-3) / (peaks["hbm_gbs"] * 1e9)}
+    step["binding"] = "tensor" if step["tensor_frac"] > step["hbm_frac"] else "hbm"
+    step["binding_frac"] = max(step["tensor_frac"], step["hbm_frac"])
+    return roof, step
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        host = oracle_args(inp)
-        rate, cores, n, dt = cpu_oracle_rate(cfg, host, args.cpu_seconds)
-        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n} seeded tokens of {cfg.name} (full block per token, fp64), {dt:.1f} s"}
+
+def time_e2e(run, K, W, world):
+    """The same metric through the public host-buffer entry point.  Like a
+    server that feeds successive batches, the steps rotate over three streams,
+    each with its own workspace and page-locked buffers, so one batch's
+    host<->device copies overlap another batch's kernels.  Every step still
+    copies its x in and its out / topk_idx / topk_w back inside the timed
+    region."""
+    cfg, inp, s, dev = run.cfg, run.inp, run.layer.shape, run.dev
+    lanes = []
+    NL = 3
+    for li in range(NL):
+        lanes.append(dict(
+            stream=run.stream if li == 0 else torch.cuda.Stream(dev),
+            ws=run.layer.workspace if li == 0 else api.alloc_workspace(s, dev),
+            xh=inp["x"].cpu().pin_memory(),
+            oh=torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16).pin_memory(),
+            ih=torch.empty((cfg.T, cfg.k), dtype=torch.int32).pin_memory(),
+            wh=torch.empty((cfg.T, cfg.k), dtype=torch.float32).pin_memory()))
+
+    def host_step(i):
+        L = lanes[i % NL]
+        api.moe_forward_host(s, L["xh"], inp["W_router"], inp["expert_bias"], inp["W_gate"], inp["W_up"],
+                             inp["W_down"], inp["W_shared_gate"], inp["W_shared_up"], inp["W_shared_down"],
+                             cfg.score_fn, cfg.norm_topk, cfg.route_scale, L["oh"], L["ih"], L["wh"], L["ws"],
+                             L["stream"], W_shared_gate_vec=inp.get("W_shared_gate_vec"))
+    for i in range(max(2 * NL, W)):
+        host_step(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    ends = [torch.cuda.Event(enable_timing=True) for _ in lanes]
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(lanes[0]["stream"])
+    for L in lanes[1:]:
+        L["stream"].wait_event(e0)
+    for i in range(K):
+        host_step(i)
+    for L, ev in zip(lanes, ends):
+        ev.record(L["stream"])
+    torch.cuda.synchronize()
+    barrier(world)
+    for L in lanes:
+        st_chk = api.moe_device_status(L["ws"], L["stream"])
+        if st_chk != api.MOE_OK:
+            raise RuntimeError(f"device status after e2e: {api.status_string(st_chk)}")
+    e2e_ms = max_over_ranks(max(e0.elapsed_time(ev) for ev in ends), world)
+    del lanes
+    return {"value": world * cfg.T * K / (e2e_ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": cfg.T * cfg.d * 2,
+            "d2h_bytes_per_step": cfg.T * cfg.d * 2 + cfg.T * cfg.k * 8,
+            "streams": NL, "ms_per_step": e2e_ms / K}
+
+
+def extra_workloads(args, main_name, dev, world, rank):
+    """Every other full-size workload, timed in this run the same way."""
+    res = {}
+    launches = 0
+    for name in EXTRA_WORKLOADS:
+        if name == main_name:
+            continue
+        cfg = variant_cfg(CONFIGS[name], args.variant)
+        K2 = max(args.steps, args.extra_steps)
+        run = Runner(cfg, args.variant, dev, replica_seed(cfg, rank))
+        tm = time_steps(run, K2, args.warmup, world)
+        roof, step = roofline_of(cfg, tm, K2, args.variant)
+        launches += K2 * run.launches_per_step()
+        res[name] = {"value": world * cfg.T * K2 / (tm["elapsed_ms"] / 1e3), "unit": "tokens/s",
+                     "steps": K2, "ms_per_step": tm["elapsed_ms"] / K2, "ms_per_step_median": tm["step_median_ms"],
+                     "config": config_dict(cfg, args.variant, world), "kernels_us": tm["stage_avg_us"],
+                     "roofline": roof, "step_roofline": step, "clocks": tm["clocks"],
+                     "touched_experts": tm["touched"], "expert_load": tm["expert_load"]}
+        del run
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return res, launches
+
+
+def run_ours(args, cfg):
+    world, rank, local = dist_setup(args.gpus)
+    api.load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    run = Runner(cfg, args.variant, dev, replica_seed(cfg, rank))
+    K = args.steps
+    tm = time_steps(run, K, args.warmup, world)
+    gpu_result = run.results_host() if rank == 0 and world == 1 and not args.no_cpu_baseline else None
+
+    # the host-buffer entry point runs the whole block on raw x with bf16
+    # weights: it has no caller-routing, pre-norm or FP8 form, so those
+    # variants report no e2e figure
+    e2e = None
+    if not args.no_e2e and not run.external and not cfg.prenorm and not cfg.fp8:
+        e2e = time_e2e(run, K, args.warmup, world)
+
+    value = world * cfg.T * K / (tm["elapsed_ms"] / 1e3)
+    roof, step_roof = roofline_of(cfg, tm, K, args.variant)
+    launches = K * run.launches_per_step()
+    inp = run.inp
+    del run
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    cpu = parity = None
+    if gpu_result is not None:
+        cpu, parity = cpu_baseline_leg(cfg, inp, gpu_result, args.cpu_seconds)
+    del inp
+    torch.cuda.empty_cache()
+
+    workloads, extra_launches = ({}, 0) if args.no_extra else extra_workloads(args, cfg.name, dev, world, rank)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-                "warmup": args.warmup, "ms_per_step": ms_step, "ms_per_step_median": step_median_ms,
+                "warmup": args.warmup, "ms_per_step": tm["elapsed_ms"] / K, "ms_per_step_median": tm["step_median_ms"],
                 "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) x, N(0,0.02) weights)",
-                "config": {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "E": cfg.E, "k": cfg.k,
-                           "d_ff": cfg.f, "n_shared": cfg.S, "d_ff_shared": cfg.fs, "score_fn": cfg.score_fn,
-                           "norm_topk": cfg.norm_topk, "touched_experts": touched, "expert_load": expert_load,
-                           "variant": args.variant or "base",
-                           "expert_weights": "fp8 e4m3 + ue8m0 scale per 32" if cfg.fp8 else "bf16",
-                           "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (
-                               weight_bytes(cfg) * cfg.E * 3 * cfg.f * cfg.d / 1e9),
-                           "parallelism": "replicas" if world > 1 else "single GPU"},
+                "config": config_dict(cfg, args.variant, world),
+                "touched_experts": tm["touched"], "expert_load": tm["expert_load"],
                 "roofline": roof, "step_roofline": step_roof,
-                "kernels_us": stage_avg_us, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": K * (sum(LAUNCHES_PER_STEP.values())
-                                     - (LAUNCHES_PER_STEP["route"] if external else 0)
-                                     + (1 if cfg.prenorm else 0)),
-                "clocks": clk.summary()}
+                "kernels_us": tm["stage_avg_us"], "cpu_baseline": cpu, "parity": parity, "e2e": e2e,
+                "gpu_launches": launches, "gpu_launches_other_workloads": extra_launches,
+                "clocks": tm["clocks"], "workloads": workloads}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -427,13 +547,7 @@ def run_ours(args, cfg):
 
 def main():
     args = parse()
-    cfg = CONFIGS[args.config]
-    if args.variant == "gated_shared":
-        cfg = dataclasses.replace(cfg, shared_gate=True)
-    if args.variant == "prenorm":
-        cfg = dataclasses.replace(cfg, prenorm=True)
-    if args.variant == "fp8":
-        cfg = dataclasses.replace(cfg, fp8=True)
+    cfg = variant_cfg(CONFIGS[args.config], args.variant)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

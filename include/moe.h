@@ -86,6 +86,8 @@ extern "C" {
 #define MOE_ERR_CUDA           -4   /* a CUDA runtime / driver call or a launch failed */
 #define MOE_ERR_DEVICE_TIMEOUT -5   /* a bounded device-side wait ran out (reported by moe_device_status) */
 #define MOE_ERR_SCRATCH_LIMIT  -6   /* moe_route_noalloc: T * E fp32 logits exceed its built-in 16 MiB scratch */
+#define MOE_ERR_NONFINITE      -7   /* a token's router logits, selection keys or combine weights were NaN or
+                                       infinite (reported by moe_device_status) */
 
 #define MOE_SCORE_SOFTMAX       0   /* s = softmax(l) over all E experts; expert_bias ignored */
 #define MOE_SCORE_SIGMOID       1   /* s = 1/(1+exp(-l)) */
@@ -327,7 +329,17 @@ MOE_API int moe_workspace_region(const moe_shape *shape, int region, size_t *off
 
 /* Synchronises `stream`, then returns MOE_ERR_DEVICE_TIMEOUT if a kernel of a
  * call on this workspace (since the last moe_route) gave up a bounded wait,
- * MOE_ERR_CUDA if the stream reports an error, else MOE_OK. */
+ * MOE_ERR_INVALID_ARG if routing handed to the permute step was invalid,
+ * MOE_ERR_NONFINITE if the routing step met a NaN or infinite logit,
+ * selection key or combine weight, MOE_ERR_CUDA if the stream reports an
+ * error, else MOE_OK (the first of these that applies).
+ *
+ * Non-finite inputs never make a kernel read or write out of bounds: a NaN
+ * selection key ranks below every other key (with -inf), so each token still
+ * gets k distinct experts in [0, E); its weights are whatever the arithmetic
+ * gives (NaN for an all-NaN row).  If the router GEMM gives up a bounded wait,
+ * the top-k step writes expert -1 and weight 0 for every token instead of
+ * routing on incomplete logits. */
 MOE_API int moe_device_status(const void *workspace, moe_stream_t stream);
 
 /* Routing (the moe_route step) for callers that cannot allocate device
@@ -349,8 +361,11 @@ MOE_API int moe_device_status(const void *workspace, moe_stream_t stream);
  *   different streams, or from different threads without ordering) race and
  *   give undefined results.  The array keeps the last call's contents; the
  *   call clears what must start at zero itself.
- *   A bounded device wait that runs out is recorded only inside that array:
- *   moe_device_status cannot report it for this entry point. */
+ *   A bounded device wait that runs out is recorded only inside that array,
+ *   which moe_device_status cannot read; it shows in the outputs instead:
+ *   every topk_idx is then -1 and every topk_w 0.  A NaN or infinite logit
+ *   is not reported for this entry point (the routing stays in range, as for
+ *   moe_route). */
 MOE_API int moe_route_noalloc(const moe_shape *shape, const void *x, const void *W_router,
                               const float *expert_bias, int score_fn, int norm_topk, float route_scale,
                               int32_t *topk_idx, float *topk_w, moe_stream_t stream);

@@ -23,6 +23,7 @@ MOE_ERR_WORKSPACE = -3
 MOE_ERR_CUDA = -4
 MOE_ERR_DEVICE_TIMEOUT = -5
 MOE_ERR_SCRATCH_LIMIT = -6
+MOE_ERR_NONFINITE = -7
 
 SCORE_FNS = {"softmax": 0, "sigmoid": 1, "sqrt_softplus": 2}
 

@@ -164,7 +164,7 @@ int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_
   int rc = launch_gemm(kModeRouter, g, grid, smem, st);
   if (rc != MOE_OK) return rc;
   return launch_topk(reinterpret_cast<const float*>(ws + p.logits), p.router_split, bias, p.T, p.E, p.k, score_fn,
-                     norm_topk, route_scale, topk_idx, topk_w, st);
+                     norm_topk, route_scale, topk_idx, topk_w, g.err, st);
 }
 
 int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, Wt Wg, Wt Wu, Wt Wsg, Wt Wsu, char* ws,
@@ -342,6 +342,14 @@ int check_gate_vec(const Plan& p, const void* W_shared_gate_vec) {
 
 }  // namespace
 
+// SMs of the current device, for the plan's tiling rules; 148 (a B200) when
+// no device can be queried (moe_workspace_bytes on a host without a GPU).
+static int plan_sms() {
+  DeviceInfo di;
+  if (device_info(&di) == MOE_OK && di.sms > 0) return di.sms;
+  return 148;
+}
+
 int make_plan(const moe_shape* s, Plan* p, bool f8) {
   if (!s || !p) return MOE_ERR_INVALID_ARG;
   const int T = s->T, d = s->d_model, E = s->E, k = s->k, f = s->d_ff, S = s->n_shared;
@@ -355,6 +363,8 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
   Plan q;
   std::memset(&q, 0, sizeof q);
   q.T = T; q.d = d; q.E = E; q.k = k; q.f = f; q.S = S; q.fs = fs;
+  const int sms = plan_sms();
+  const int half_sms = sms / 2;
   const double rows_per_expert = static_cast<double>(T) * k / E;
   q.nmax1 = pick_nmax(rows_per_expert);
   // Experts of 256+ rows on average: the gate/up GEMM runs on CTA pairs,
@@ -383,14 +393,14 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
   q.nwb1s = S > 0 ? ceil_div(fs, rows1) : 0;
   q.nwb2 = ceil_div(d, rows2);
   // Router: runs of up to 128 tokens (their fp32 logit sums live in
-  // registers) when that still gives every SM of a B200 a unit; else runs of
-  // 64 or narrower while most SMs stay busy.
+  // registers) when that still gives every SM a unit; else runs of 64 or
+  // narrower while most SMs stay busy.
   q.nmax_r = 16;
-  if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, 128) >= 148) {
+  if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, 128) >= sms) {
     q.nmax_r = 128;
   } else {
     for (int n = 64; n >= 16; n >>= 1) {
-      if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, n) >= 74) {
+      if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, n) >= half_sms) {
         q.nmax_r = n;
         break;
       }
@@ -402,8 +412,8 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
     const int base = q.nwbE * ceil_div(q.Tp, q.nmax_r);
     const int KB = d / kTileK;
     int split = 1;
-    if (base < 74) {
-      split = 148 / base;
+    if (base < half_sms) {
+      split = sms / base;
       if (split > kMaxRouterSplit) split = kMaxRouterSplit;
       if (split > KB) split = KB;
       if (split < 1) split = 1;
@@ -419,7 +429,7 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
         const int kbs = ceil_div(KB, sp);
         const int ns = ceil_div(KB, kbs);
         const long long units = static_cast<long long>(q.nwbE) * ceil_div(q.Tp, n) * ns;
-        const long long per_sm = (units + 147) / 148;
+        const long long per_sm = (units + sms - 1) / sms;
         const double ingest = static_cast<double>(per_sm) * (kTileRows + n) * kbs * kTileK * 2;
         const double partials = static_cast<double>(ns - 1) * T * E * 4 * 2;
         return ingest / 47e9 + partials / 6.5e12;
@@ -529,6 +539,7 @@ const char* moe_status_string(int status) {
     case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a bounded device-side wait ran out";
     case MOE_ERR_SCRATCH_LIMIT:
       return "MOE_ERR_SCRATCH_LIMIT: T * E fp32 logits exceed the 16 MiB built-in scratch of moe_route_noalloc";
+    case MOE_ERR_NONFINITE: return "MOE_ERR_NONFINITE: NaN or infinite router logits, selection keys or weights";
     default: return "unknown status";
   }
 }
@@ -838,6 +849,7 @@ int moe_device_status(const void* workspace, moe_stream_t stream) {
   if (cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
   if (word & kDevErrTimeout) return MOE_ERR_DEVICE_TIMEOUT;
   if (word & (kDevErrBadRouting | kDevErrPlanMismatch)) return MOE_ERR_INVALID_ARG;
+  if (word & kDevErrNonFinite) return MOE_ERR_NONFINITE;
   return MOE_OK;
 }
 
@@ -945,5 +957,5 @@ extern "C" int moe_route_noalloc(const moe_shape* shape, const void* x, const vo
   const int grid = p.router_units < di.sms ? p.router_units : di.sms;
   if ((rc = launch_gemm(kModeRouter, g, grid, smem, st)) != MOE_OK) return rc;
   return launch_topk(logits, p.router_split, expert_bias, p.T, p.E, p.k, score_fn, norm_topk, route_scale, topk_idx,
-                     topk_w, st);
+                     topk_w, err, st);
 }

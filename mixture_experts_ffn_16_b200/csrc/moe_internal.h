@@ -156,8 +156,12 @@ size_t gemm_f8_smem_bytes(int mode, int nmax, int* stages, int* tok_stages, int*
 int launch_gemm_pair(int mode, const GemmParams& prm, int grid, size_t smem, cudaStream_t st);
 size_t gemm_pair_smem_bytes(int mode, int nmax, int* stages);
 
+// err: the error word of this call.  If the router GEMM recorded a timeout
+// there, every token gets expert -1 and weight 0; NaN or infinite keys or
+// weights set kDevErrNonFinite.
 int launch_topk(const float* logits, int nsplit, const float* bias, int T, int E, int k, int score_fn,
-                int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w, cudaStream_t st);
+                int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w, uint32_t* err,
+                cudaStream_t st);
 
 int launch_permute(const Plan& p, const int32_t* topk_idx, const float* topk_w, char* ws,
                    cudaStream_t st);

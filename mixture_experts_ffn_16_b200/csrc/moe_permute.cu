@@ -5,9 +5,11 @@
 //             per-expert histogram.
 //   scan    : one block: per expert, exclusive prefix over blocks (-> each
 //             block's offset inside the expert's segment) and the expert's
-//             count; then exclusive scans over experts of the padded segment
-//             sizes and of the GEMM work-unit counts; writes the work lists
-//             and fills the padding rows.
+//             count; then an exclusive scan over experts of the padded segment
+//             sizes (rows stay in expert order), a rank of every expert by
+//             padded rows (largest first), exclusive scans in rank order of
+//             the GEMM work-unit counts; writes the work lists (largest
+//             expert first) and fills the padding rows.
 //   scatter : recomputes the masks (each of the ceil(k/2) CTAs of a block
 //             places two slots of its tokens); a (token, slot) pair's row is
 //             segment start + block offset + popcount of the lower lanes of
@@ -111,6 +113,7 @@ __device__ int3 block_exclusive_scan3(int3 v, int3* total) {
   __syncthreads();
   const int3 base = warp > 0 ? wsum[warp - 1] : make_int3(0, 0, 0);
   *total = wsum[kScanThreads / 32 - 1];
+  __syncthreads();   // wsum may be reused by the next call
   return make_int3(base.x + inc.x - v.x, base.y + inc.y - v.y, base.z + inc.z - v.z);
 }
 
@@ -130,12 +133,16 @@ struct ScanArgs {
 };
 
 __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) {
+  // Padded rows of every expert, then (by rank) its unit counts and their
+  // exclusive offsets: the work lists run largest expert first.
+  __shared__ __align__(16) int s_key[kMaxE];
+  __shared__ int s_u1[kMaxE], s_u2[kMaxE];
   chain_wait();
   // Experts per thread, contiguous: one up to E = 1024, else two.
   constexpr int kPer = (kMaxE + kScanThreads - 1) / kScanThreads;
   const int per = a.E > kScanThreads ? kPer : 1;
-  int cnt[kPer], pad[kPer], u1[kPer], u2[kPer];
-  int sp = 0, s1 = 0, s2 = 0;
+  int cnt[kPer], pad[kPer], u1[kPer], u2[kPer], rank[kPer];
+  int sp = 0;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = (i < per) ? threadIdx.x * per + i : a.E;
@@ -160,16 +167,66 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) 
     pad[i] = (c + a.rowpad - 1) / a.rowpad * a.rowpad;
     u1[i] = (pad[i] + a.nmax1 - 1) / a.nmax1 * a.nwb1;
     u2[i] = (pad[i] + a.nmax2 - 1) / a.nmax2 * a.nwb2;
+    if (e < a.E) s_key[e] = pad[i];
     sp += pad[i];
-    s1 += u1[i];
-    s2 += u2[i];
   }
   int3 tot;
-  const int3 ex = block_exclusive_scan3(make_int3(sp, s1, s2), &tot);
-  const int tot_rows = tot.x, tot1 = tot.y, tot2 = tot.z;
+  const int3 ex = block_exclusive_scan3(make_int3(sp, 0, 0), &tot);
+  const int tot_rows = tot.x;
+  // Rank of each expert in the work lists: more padded rows first, then the
+  // lower expert index (a strict order, so ranks are 0..E-1).  Each work
+  // list then starts with the biggest experts, so the units of the last
+  // rounds over the SMs are the smallest.  Rows keep the expert order.
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = (i < per) ? threadIdx.x * per + i : a.E;
+    rank[i] = 0;
+    if (e < a.E) {
+      int r = 0;
+      const int key = pad[i];
+      const int E4 = a.E & ~3;
+      for (int e2 = 0; e2 < E4; e2 += 4) {
+        const int4 k4 = *reinterpret_cast<const int4*>(s_key + e2);
+        r += (k4.x > key || (k4.x == key && e2 < e)) + (k4.y > key || (k4.y == key && e2 + 1 < e)) +
+             (k4.z > key || (k4.z == key && e2 + 2 < e)) + (k4.w > key || (k4.w == key && e2 + 3 < e));
+      }
+      for (int e2 = E4; e2 < a.E; ++e2) r += (s_key[e2] > key || (s_key[e2] == key && e2 < e));
+      rank[i] = r;
+      s_u1[r] = u1[i];
+      s_u2[r] = u2[i];
+    }
+  }
+  __syncthreads();
+  // Unit offsets in rank order (thread i owns ranks i*per ..).
+  int r1[kPer], r2[kPer];
+  int s1 = 0, s2 = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int r = (i < per) ? threadIdx.x * per + i : a.E;
+    r1[i] = r < a.E ? s_u1[r] : 0;
+    r2[i] = r < a.E ? s_u2[r] : 0;
+    s1 += r1[i];
+    s2 += r2[i];
+  }
+  int3 utot;
+  const int3 uex = block_exclusive_scan3(make_int3(0, s1, s2), &utot);
+  const int tot1 = utot.y, tot2 = utot.z;
+  __syncthreads();   // every s_u1 / s_u2 read above is done
+  {
+    int o1 = uex.y, o2 = uex.z;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int r = (i < per) ? threadIdx.x * per + i : a.E;
+      if (r < a.E) {
+        s_u1[r] = o1;
+        s_u2[r] = o2;
+      }
+      o1 += r1[i];
+      o2 += r2[i];
+    }
+  }
+  __syncthreads();
   int ro = ex.x;
-  int o1 = a.shared_units1 + ex.y;
-  int o2 = a.shared_units2 + ex.z;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = (i < per) ? threadIdx.x * per + i : a.E;
@@ -180,6 +237,8 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) 
         a.perm[ro + r] = 0;
         a.roww[ro + r] = 0.0f;
       }
+      const int o1 = a.shared_units1 + s_u1[rank[i]];
+      const int o2 = a.shared_units2 + s_u2[rank[i]];
       // gate/up units: (e, wb, chunk), chunks inner so that consecutive units share a weight tile
       const int nch1 = (pad[i] + a.nmax1 - 1) / a.nmax1;
       for (int wb = 0; wb < a.nwb1; ++wb)
@@ -191,8 +250,6 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) 
           a.units2[o2 + wb * nch2 + c] = make_int4(e, wb, ro + c * a.nmax2, min(a.nmax2, pad[i] - c * a.nmax2));
     }
     ro += pad[i];
-    o1 += u1[i];
-    o2 += u2[i];
   }
   // Shared-expert units (first in each list).
   const int nch1s = (a.Tp + a.nmax1 - 1) / a.nmax1;

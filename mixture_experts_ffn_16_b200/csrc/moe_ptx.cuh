@@ -17,6 +17,7 @@ enum : uint32_t {
   kDevErrTimeout = 1u,        // a bounded wait ran out
   kDevErrBadRouting = 2u,     // topk_idx held an expert out of range or a repeated expert
   kDevErrPlanMismatch = 4u,   // an expert GEMM met work lists built for the other weight format
+  kDevErrNonFinite = 8u,      // a token's router logits, selection keys or combine weights were NaN / inf
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -136,6 +136,45 @@ def test_invalid_routing_is_reported_not_faulted():
     assert api.moe_device_status(ws) == api.MOE_ERR_INVALID_ARG
 
 
+def test_nonfinite_router_inputs_stay_in_range_and_are_reported(case):
+    """A token row of x that is all NaN, and a NaN expert bias: every token
+    still gets k distinct experts in [0, E) (a NaN key ranks with -inf, below
+    every other key, ties to the lower index), the other tokens' routing and
+    outputs are those of a run without the NaN row, and moe_device_status
+    reports MOE_ERR_NONFINITE."""
+    inp, layer = case
+    T, E, k = CFG.T, CFG.E, CFG.k
+    bad_t = 5
+    x_clean = inp["x"].clone()
+    x_clean[bad_t] = 0.0
+    o_ref, i_ref, w_ref = [t.clone() for t in layer(x_clean)]
+    assert api.moe_device_status(layer.workspace) == api.MOE_OK
+    x_nan = x_clean.clone()
+    x_nan[bad_t] = float("nan")
+    o, i, w = [t.clone() for t in layer(x_nan)]
+    assert api.moe_device_status(layer.workspace) == api.MOE_ERR_NONFINITE
+    idx = i.cpu().numpy()
+    assert ((idx >= 0) & (idx < E)).all()
+    assert all(len(set(r)) == k for r in idx.tolist())
+    assert idx[bad_t].tolist() == list(range(k))          # all keys NaN: the lowest indices
+    keep = torch.ones(T, dtype=torch.bool)
+    keep[bad_t] = False
+    assert torch.equal(i[keep.cuda()], i_ref[keep.cuda()])
+    assert torch.equal(w[keep.cuda()], w_ref[keep.cuda()])
+    assert torch.equal(o[keep.cuda()].view(torch.int16), o_ref[keep.cuda()].view(torch.int16))
+    # a NaN selection bias: that expert ranks last for every token
+    bias = inp["expert_bias"].clone()
+    bias[3] = float("nan")
+    api.moe_route(layer.shape, x_clean, inp["W_router"], bias, CFG.score_fn, CFG.norm_topk, CFG.route_scale,
+                  layer.topk_idx, layer.topk_w, layer.workspace)
+    assert api.moe_device_status(layer.workspace) == api.MOE_ERR_NONFINITE
+    idx = layer.topk_idx.cpu().numpy()
+    assert ((idx >= 0) & (idx < E)).all() and not (idx == 3).any()
+    assert torch.isfinite(layer.topk_w).all()
+    layer()
+    assert api.moe_device_status(layer.workspace) == api.MOE_OK
+
+
 def test_status_ok_then_bounded_wait_timeout_then_usable(case):
     inp, layer = case
     layer()

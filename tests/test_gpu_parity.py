@@ -14,7 +14,7 @@ import torch
 from mixture_experts_ffn_16_b200 import api
 from mixture_experts_ffn_16_b200.inputs import CONFIGS, MoEConfig, make_inputs, oracle_args
 
-from parity_util import check_parity
+from parity_util import check_parity, check_routing
 
 pytestmark = pytest.mark.gpu
 
@@ -66,9 +66,10 @@ MEDIUM = [
 ]
 
 
-def test_tiny_workload_every_token(oracle_mod):
+def test_tiny_workload_every_token(oracle_mod, parity_log):
     rep, _ = parity_case(oracle_mod, CONFIGS["tiny"])
     assert rep["tokens"] == 64
+    parity_log.append(dict(case="tiny", check="block", **rep))
 
 
 @pytest.mark.parametrize("cfg", MEDIUM, ids=lambda c: c.name)
@@ -97,9 +98,15 @@ def _sample(T, n, seed):
     return np.sort(rng.choice(T, size=min(n, T), replace=False)).astype(np.int32)
 
 
-@pytest.mark.parametrize("name,n_tok", [("prefill_softmax", 384), ("prefill_sigmoid", 128),
-                                        ("decode_sqrt_softplus", 64), ("large_imbalanced", 48)])
-def test_full_size_workloads_sampled(oracle_mod, name, n_tok):
+# Tokens whose outputs are checked at full size: every token of prefill_softmax
+# and decode, a seeded 1,024-token sample of the two largest workloads.  The
+# routing (indices and weights) is checked on every token of every workload.
+FULL_SIZE = [("prefill_softmax", None), ("prefill_sigmoid", 1024), ("decode_sqrt_softplus", None),
+             ("large_imbalanced", 1024)]
+
+
+@pytest.mark.parametrize("name,n_tok", FULL_SIZE, ids=[n for n, _ in FULL_SIZE])
+def test_full_size_workloads(oracle_mod, parity_log, name, n_tok):
     cfg = CONFIGS[name]
     _need_gpu()
     inp = make_inputs(cfg, device="cuda")
@@ -107,7 +114,6 @@ def test_full_size_workloads_sampled(oracle_mod, name, n_tok):
     # properties at any size: finite output, valid routing, weights sum to route_scale
     assert np.isfinite(out).all()
     assert ((idx >= 0) & (idx < cfg.E)).all()
-    assert all(len(set(r)) == cfg.k for r in idx[: min(cfg.T, 4096)].tolist())
     if cfg.norm_topk:
         np.testing.assert_allclose(w.sum(1), cfg.route_scale, rtol=1e-5)
     counts = np.bincount(idx.ravel(), minlength=cfg.E)
@@ -120,10 +126,18 @@ def test_full_size_workloads_sampled(oracle_mod, name, n_tok):
         print(name, "expert load max/min", ratio, "max", counts.max(), "min nonzero", nz.min(),
               "empty", int((counts == 0).sum()))
         assert ratio > 10
-    tokens = _sample(cfg.T, n_tok, seed=cfg.seed + 100)
+    del layer
     host = oracle_args(inp)
-    rep = check_parity(oracle_mod, cfg, host, out[tokens], idx[tokens], w[tokens], tokens=tokens)
-    print(name, rep)
+    del inp
+    route = check_routing(oracle_mod, cfg, host, idx, w)
+    assert route["tokens"] == cfg.T
+    parity_log.append(dict(case=name, check="routing", **route))
+    tokens = None if n_tok is None else _sample(cfg.T, n_tok, seed=cfg.seed + 100)
+    sel = slice(None) if tokens is None else tokens
+    rep = check_parity(oracle_mod, cfg, host, out[sel], idx[sel], w[sel], tokens=tokens)
+    assert rep["tokens"] == (cfg.T if n_tok is None else n_tok)
+    parity_log.append(dict(case=name, check="block", **rep))
+    print(name, route, rep)
 
 
 GATED = [

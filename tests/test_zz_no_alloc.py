@@ -5,16 +5,19 @@ allocator).  Its scratch is an array built into the library, so the caller
 passes only inputs and outputs.
 
 Checked through the C ABI against moe_route (the workspace entry point) on
-two calls in a row; also that a shape beyond the built-in scratch is refused
-before anything is enqueued.  This file is collected last on purpose."""
+two calls in a row, and against the fp64 oracle by the same index, near-tie
+and weight rules as moe_route; also a shape whose partial logits would not fit
+the built-in scratch (the call then sums fewer slices of d, in another order),
+and that a shape beyond the built-in scratch is refused before anything is
+enqueued.  This file is collected last on purpose."""
 import numpy as np
 import pytest
 import torch
 
 from mixture_experts_ffn_16_b200 import api
-from mixture_experts_ffn_16_b200.inputs import CONFIGS, MoEConfig, make_inputs
+from mixture_experts_ffn_16_b200.inputs import CONFIGS, MoEConfig, bf16_bits, make_inputs, oracle_args
 
-from parity_util import W_ATOL, W_RTOL
+from parity_util import W_ATOL, W_RTOL, check_routing
 
 pytestmark = pytest.mark.gpu
 
@@ -36,7 +39,7 @@ def _route_with_workspace(cfg, inp):
     MoEConfig("noalloc_sigmoid_bias", T=777, d=512, E=96, k=6, f=128, S=1, fs=128, score_fn="sigmoid",
               bias_std=0.1, route_scale=2.5, seed=41),
 ], ids=lambda c: c.name)
-def test_noalloc_route_matches_workspace_route_twice(cfg):
+def test_noalloc_route_matches_workspace_route_twice(oracle_mod, cfg):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     api.load()
@@ -52,6 +55,35 @@ def test_noalloc_route_matches_workspace_route_twice(cfg):
         got_idx, got_w = idx.cpu().numpy(), w.cpu().numpy()
         assert np.array_equal(got_idx, ref_idx)
         np.testing.assert_allclose(got_w, ref_w, rtol=W_RTOL, atol=W_ATOL)
+    rep = check_routing(oracle_mod, cfg, oracle_args(inp), got_idx, got_w)
+    print(cfg.name, rep)
+
+
+def test_noalloc_route_with_fewer_slices_matches_oracle(oracle_mod, parity_log):
+    """prefill_sigmoid: T * E fp32 logits (12.6 MB) fit the 16 MiB scratch, but
+    the workspace plan's two slices of d (25 MB of partial logits) do not, so
+    the call sums the logits over one slice: a different fp32 summation order
+    than moe_route, checked against the oracle by the near-tie rule."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    api.load()
+    cfg = CONFIGS["prefill_sigmoid"]
+    shape = api.shape_of(cfg)
+    off, nbytes = api.moe_workspace_region(shape, "logits")
+    assert nbytes > 16 * 2**20 >= cfg.T * cfg.E * 4         # the branch that cuts the slices
+    inp = {n: t for n, t in make_inputs(cfg, device="cuda").items()
+           if n in ("x", "W_router", "expert_bias")}
+    for _ in range(2):
+        idx = torch.full((cfg.T, cfg.k), -7, dtype=torch.int32, device="cuda")
+        w = torch.full((cfg.T, cfg.k), -7.0, dtype=torch.float32, device="cuda")
+        api.moe_route_noalloc(shape, inp["x"], inp["W_router"], inp["expert_bias"], cfg.score_fn,
+                              cfg.norm_topk, cfg.route_scale, idx, w)
+        torch.cuda.synchronize()
+        host = {"x": bf16_bits(inp["x"]), "W_router": bf16_bits(inp["W_router"]),
+                "expert_bias": inp["expert_bias"].cpu().numpy()}
+        rep = check_routing(oracle_mod, cfg, host, idx.cpu().numpy(), w.cpu().numpy())
+        assert rep["tokens"] == cfg.T
+    parity_log.append(dict(case="prefill_sigmoid_noalloc", check="routing", **rep))
 
 
 def test_noalloc_route_refuses_shapes_beyond_its_scratch():
