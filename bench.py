@@ -59,6 +59,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="large_imbalanced", choices=list(CONFIGS))
+    ap.add_argument("--shape", default="", help="T,d,E,k,f,S,fs: a custom workload instead of --config "
+                    "(softmax router unless --score; seeded like the others; for small ncu captures)")
+    ap.add_argument("--score", default="softmax", choices=["softmax", "sigmoid", "sqrt_softplus"])
+    ap.add_argument("--bias-std", type=float, default=0.0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
@@ -545,9 +549,17 @@ def run_ours(args, cfg):
     return 0
 
 
+def custom_cfg(args):
+    """The workload of --shape: the given sizes, seeded N(0,1) x and N(0,0.02) weights."""
+    from mixture_experts_ffn_16_b200.inputs import MoEConfig
+    T, d, E, k, f, S, fs = (int(v) for v in args.shape.split(","))
+    return MoEConfig(f"custom_T{T}_d{d}_E{E}_k{k}_f{f}_S{S}_fs{fs}", T=T, d=d, E=E, k=k, f=f, S=S, fs=fs,
+                     score_fn=args.score, bias_std=args.bias_std, seed=5)
+
+
 def main():
     args = parse()
-    cfg = variant_cfg(CONFIGS[args.config], args.variant)
+    cfg = variant_cfg(custom_cfg(args) if args.shape else CONFIGS[args.config], args.variant)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)
