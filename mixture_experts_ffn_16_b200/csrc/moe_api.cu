@@ -106,6 +106,20 @@ bool map_rows(CUtensorMap* m, const void* ptr, int K, int rows, int box_rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// An expert GEMM's output rows [rows, cols] bf16, stored by the epilogue in
+// boxes of 32 columns x 16 rows (64-byte row segments, no swizzle).
+bool map_out(CUtensorMap* m, const void* ptr, int cols, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {32, 16};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The four token-row maps of one source: boxes of 16, 32, 64 and 128 rows.
 bool map_rows_set(CUtensorMap (&m)[4], const void* ptr, int K, int rows) {
   for (int b = 0; b < 4; ++b)
@@ -186,6 +200,12 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, Wt Wg, Wt Wu
     g.mapS[3] = g.mapS[1];
   }
   copy_set(g.mapB[1], g.mapB[0]);
+  if (!map_out(&g.mapO[0], ws + p.Hr, p.f, p.Rcap)) return MOE_ERR_CUDA;
+  if (p.S > 0) {
+    if (!map_out(&g.mapO[1], ws + p.Hs, p.fs, p.S * p.Tp)) return MOE_ERR_CUDA;
+  } else {
+    g.mapO[1] = g.mapO[0];
+  }
   g.units = reinterpret_cast<const int4*>(ws + p.units1);
   g.plan_tag_dev = reinterpret_cast<const int*>(ws + p.nunits) + 3;
   g.plan_tag = plan_tag(p);
@@ -240,6 +260,12 @@ int run_down(const Plan& p, const DeviceInfo& di, Wt Wd, Wt Wsd, char* ws, cudaS
   g.mapA[3] = g.mapA[2];
   g.mapS[1] = g.mapS[0];
   g.mapS[3] = g.mapS[2];
+  if (!map_out(&g.mapO[0], ws + p.Yr, p.d, p.Rcap)) return MOE_ERR_CUDA;
+  if (p.S > 0) {
+    if (!map_out(&g.mapO[1], ws + p.Ys, p.d, p.S * p.Tp)) return MOE_ERR_CUDA;
+  } else {
+    g.mapO[1] = g.mapO[0];
+  }
   g.units = reinterpret_cast<const int4*>(ws + p.units2);
   g.plan_tag_dev = reinterpret_cast<const int*>(ws + p.nunits) + 3;
   g.plan_tag = plan_tag(p);

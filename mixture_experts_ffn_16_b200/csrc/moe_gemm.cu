@@ -58,7 +58,11 @@ __host__ __device__ constexpr int threads_of(int mode, bool f8 = false) {
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kATileBytes = kTileRows * 128;   // 128 weight rows x 64 bf16
-constexpr int kEpiBytes = 8192;                      // transpose staging, shared by the epilogue warps
+constexpr int kEpiBytes = 8192;                      // transpose staging of the CTA-pair kernel's epilogue warps
+// Epilogue staging of the single-CTA kernel: 2 KB per warp (router: one fp32
+// transpose buffer; expert GEMMs: two 1 KB slots that alternate, so a slot
+// is refilled while the tensor store of the other is in flight).
+__host__ __device__ constexpr int epi_bytes_of(int mode) { return 2048 * epi_warps_of(mode); }
 constexpr int kMaxStages = 8;
 constexpr int kSmemAlign = 1024;
 constexpr int kSmemTail = 768;                       // barriers, TMEM slot, abort flag
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
   uint8_t* tokring = smem + static_cast<size_t>(S) * stage_bytes;
   uint8_t* raw = tokring + static_cast<size_t>(TS) * tok_bytes;
   uint8_t* epi = raw + static_cast<size_t>(R) * raw_stage_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(epi + kEpiBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi + epi_bytes_of(MODE));
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + kMaxTmemBufs;
@@ -684,7 +688,7 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
   } else if (warp >= 2 && warp < 2 + epi_warps_of(MODE)) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                       // TMEM lane quarter this warp may read
-    uint8_t* stg = epi + (warp - 2) * (kEpiBytes / epi_warps_of(MODE));
+    uint8_t* stg = epi + (warp - 2) * 2048;
     if constexpr (MODE == kModeRouter) {
       // Router: sum the drained partial logits in fp32 registers, then write
       // logits[t, e] (thread = expert row, column = token).
@@ -771,6 +775,7 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
       }
     } else {
       uint32_t ucount = 0;
+      uint32_t ech = 0;                 // chunks stored by this warp (staging slot = ech & 1)
       for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
         const Unit un = get_unit<MODE>(p, u);
         const bool sh = (MODE != kModeRouter) && un.g >= p.E;
@@ -800,13 +805,16 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
         const int feat0 = un.wb * kWbRows + h * kTileRows + 32 * q;   // first weight row of this warp
         const int wrows = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
         if (feat0 < wrows) {
-          const int ld = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
-          __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(sh ? p.out_s : p.out_r);
           const size_t rbase = (sh ? static_cast<size_t>(sidx) * p.Tp : 0) + static_cast<size_t>(un.row0);
-          // 16 columns: fp32 math, bf16, transpose through shared memory,
-          // 16-byte stores of 64-byte row segments.
+          // 16 columns: fp32 math, bf16, transposed into a staging slot as
+          // 16 rows x 32 features (64-byte rows), which one tensor store
+          // writes to rows rbase + c .. + 15, features feat0 .. + 31.
+          const CUtensorMap* omap = &p.mapO[sh ? 1 : 0];
           auto emit = [&](const uint32_t (&A)[16], const uint32_t (&B)[16], int c, float wsel) {
-            __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
+            uint8_t* slot = stg + (ech & 1u) * 1024u;
+            if (lane == 0) bulk_wait_group_read<1>();   // the store from this slot two chunks ago has read it
+            __syncwarp();
+            __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(slot);
             if (MODE == kModeGateUp) {
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
@@ -821,15 +829,13 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
                 sb[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(A[i]) * w);
               }
             }
+            fence_proxy_async_smem();                     // these writes -> the tensor store's reads
             __syncwarp();
-#pragma unroll
-            for (int rep = 0; rep < 2; ++rep) {
-              const int cc = lane + 32 * rep;
-              const int tok = cc >> 2, part = cc & 3;
-              const uint4 v = *reinterpret_cast<const uint4*>(stg + tok * 64 + part * 16);
-              *reinterpret_cast<uint4*>(outp + (rbase + c + tok) * ld + feat0 + part * 8) = v;
+            if (lane == 0) {
+              tma_store_2d(omap, smem_u32(slot), feat0, static_cast<int>(rbase) + c);
+              bulk_commit_group();
             }
-            __syncwarp();
+            ++ech;
           };
           // Two register sets: the TMEM load of the next 16 columns is in
           // flight while the current ones are converted and stored.  This
@@ -865,6 +871,7 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
         if (lane == 0) mbar_arrive(&tempty[buf]);
         ++ucount;
       }
+      if (lane == 0) bulk_wait_group_all();        // every output row written before the block leaves
     }
     }
   tc_fence_before();
@@ -1247,7 +1254,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
 size_t gemm_smem_bytes(int mode, int nmax, int* stages) {
   const int NA = (mode == kModeRouter) ? 1 : 2;
   const size_t stage_bytes = NA * static_cast<size_t>(kATileBytes) + static_cast<size_t>(nmax) * 128;
-  const size_t fixed = kSmemAlign + kEpiBytes + kSmemTail;
+  const size_t fixed = kSmemAlign + epi_bytes_of(mode) + kSmemTail;
   const size_t budget = 232448;   // sm_100 opt-in maximum per block
   int s = static_cast<int>((budget - fixed) / stage_bytes);
   if (s > kMaxStages) s = kMaxStages;
@@ -1291,9 +1298,8 @@ size_t gemm_f8_smem_bytes(int mode, int nmax, int* stages, int* tok_stages, int*
   const size_t stage_bytes = 0;   // widened tiles live in tensor memory
   const size_t tok_bytes = static_cast<size_t>(nmax) * 128;
   const size_t raw_stage = NA * static_cast<size_t>(kRawTile);
-  const size_t fixed = kSmemAlign + kEpiBytes + kSmemTail;
+  const size_t fixed = kSmemAlign + epi_bytes_of(mode) + kSmemTail;
   const size_t budget = 232448;
-  (void)mode;
   const int s = kAStages;
   int ts = static_cast<int>(65536 / tok_bytes);   // 64 KB of token tiles
   if (ts < 2) ts = 2;
