@@ -74,22 +74,18 @@ def block_cost(cfg, touched=None):
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch, from
-# the committed ncu capture of the three GEMMs of one prefill_softmax step.
-# Each figure holds for the moe_gemm.cu revisions listed with it (sha256
-# prefix of the source without comments, see _gemm_source_sha):
-#   5335669b4bc0657e  the captured revision;
-#   123a73c1a8dd1b41  differs from it only in host code: the launchers cache
-#                     the kernels' shared-memory limits under a lock.  The
-#                     kernels and their launch configuration are the ones
-#                     captured.
-# The router's figure holds for the captured revision only: the router's
-# tiling (run width, K slices) changed after the capture.
-_CAPTURED = "5335669b4bc0657e"
-_HOST_ONLY_CHANGE = "123a73c1a8dd1b41"
+# the committed ncu captures (profiles/): the three GEMMs of one
+# prefill_softmax step, captured at full size.  Each figure holds for the
+# moe_gemm.cu revision listed with it (sha256 prefix of the source without
+# comments, see _gemm_source_sha).  The other workloads are too large for a
+# full-counter capture; their reduced-size captures (profiles/) do not scale
+# to a full launch in proportion (token-row reuse depends on k and E), so
+# their traffic is reported as unknown (None).
+_CAPTURED = "60e5b57f8589feb3"
 NCU_TRAFFIC = {
     ("prefill_softmax", "route"): (17.9e6, {_CAPTURED}),
-    ("prefill_softmax", "gate_up"): (1108.3e6, {_CAPTURED, _HOST_ONLY_CHANGE}),
-    ("prefill_softmax", "down"): (747.3e6, {_CAPTURED, _HOST_ONLY_CHANGE}),
+    ("prefill_softmax", "gate_up"): (1109.9e6, {_CAPTURED}),
+    ("prefill_softmax", "down"): (751.6e6, {_CAPTURED}),
 }
 
 
