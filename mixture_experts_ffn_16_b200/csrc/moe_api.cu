@@ -393,10 +393,12 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
   const int half_sms = sms / 2;
   const double rows_per_expert = static_cast<double>(T) * k / E;
   q.nmax1 = pick_nmax(rows_per_expert);
-  // Experts of 256+ rows on average: the gate/up GEMM runs on CTA pairs,
-  // each CTA loading half of every token tile (runs then come in multiples of
-  // 32).  Below that, and for the down GEMM (measured), the pair's cross-CTA
-  // handshakes cost more than the halved token loads save.
+  // Experts of 256+ rows on average: both expert GEMMs run on CTA pairs.
+  // Gate/up: each CTA loads half of every token tile (runs then come in
+  // multiples of 32).  Down: each CTA holds one 256-column accumulator
+  // instead of two, so tensor memory takes two buffers and a unit's epilogue
+  // overlaps the next unit's MMAs.  Below 256 rows the pair's cross-CTA
+  // handshakes cost more than they save (measured).
   const int pair_bf16 = (q.nmax1 >= 64 && rows_per_expert >= 256.0) ? 1 : 0;
   // FP8 expert weights: single CTAs, token runs of at most 128 (their
   // accumulators share tensor memory with the widened weight tiles).  The
@@ -404,7 +406,7 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
   if (f8 && q.nmax1 > 128) q.nmax1 = 128;
   q.nmax2 = q.nmax1;
   q.pair1 = f8 ? 0 : pair_bf16;
-  q.pair2 = 0;
+  q.pair2 = f8 ? 0 : pair_bf16;
   q.rowpad = pair_bf16 ? 2 * kRowPad : kRowPad;
   // Experts that fit one token run on average read each weight tile once.
   q.weights_evict_first = rows_per_expert <= 0.75 * q.nmax1 ? 1 : 0;

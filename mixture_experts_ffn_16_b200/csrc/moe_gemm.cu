@@ -894,8 +894,9 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
 // tile that a single CTA would: the token bytes that stream into the SMs are
 // halved for the same weight bytes.
 //   gate/up : wb = 256-row block of f; A tiles per CTA: gate rows, up rows.
-//   down    : wb = 512-row block of d; A tiles per CTA: its 128 rows of the
-//             two 256-row halves (two accumulators).
+//   down    : wb = 256-row block of d; A tile per CTA: its 128 rows (one
+//             256-column accumulator per CTA, so tensor memory holds two
+//             buffers and the epilogue of one unit overlaps the next's MMAs).
 // The leader CTA (rank 0) issues the MMAs; loads of both CTAs complete on the
 // leader's stage barrier (cta_group::2 tensor loads, no multicast); the
 // leader's commits arrive on the barrier at the same offset in both CTAs.
