@@ -187,7 +187,8 @@ int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, Wt Wg, Wt Wu
   std::memset(&g, 0, sizeof g);
   const bool f8 = Wg.s != nullptr;
   if (!map_weight_operand(&g.mapA[0], &g.mapS[0], Wg, p.d, p.f, p.E) ||
-      !map_weight_operand(&g.mapA[1], &g.mapS[1], Wu, p.d, p.f, p.E) || !map_rows_set(g.mapB[0], x, p.d, p.T))
+      !map_weight_operand(&g.mapA[1], &g.mapS[1], Wu, p.d, p.f, p.E) || !map_rows_set(g.mapB[0], x, p.d, p.T) ||
+      !map_rows(&g.mapX, x, p.d, p.T, 1))
     return MOE_ERR_CUDA;
   if (p.S > 0) {
     if (!map_weight_operand(&g.mapA[2], &g.mapS[2], Wsg, p.d, p.fs, p.S) ||

@@ -23,9 +23,9 @@
 //   epilogue    4 (router) or 8 warps: tcgen05.ld -> fp32 math (SiLU*, weight
 //               scale) -> bf16 -> transpose through shared memory -> 16-byte
 //               stores of whole row segments.
-//   gather      gate/up: 4 warps copy the unit's token rows of x (by perm) with
-//               cp.async straight into the swizzled tile; no permuted copy of
-//               x is ever made.
+//   gather      gate/up: 4 warps copy the unit's token rows of x (by perm)
+//               straight into the swizzled tile (cp.async; CTA pairs: 4-row
+//               tensor gathers); no permuted copy of x is ever made.
 //   FP8 forms   block-scaled FP8 weights: converter warps widen landed FP8
 //               tiles into tensor memory (see moe_gemm_kernel<MODE, true>).
 //
@@ -898,10 +898,14 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
 //             256-column accumulator per CTA, so tensor memory holds two
 //             buffers and the epilogue of one unit overlaps the next's MMAs).
 // The leader CTA (rank 0) issues the MMAs; loads of both CTAs complete on the
-// leader's stage barrier (cta_group::2 tensor loads, no multicast); the
-// leader's commits arrive on the barrier at the same offset in both CTAs.
-// The second CTA's gathered token rows (cp.async) complete on its own barrier
-// and are forwarded to the leader by its otherwise idle MMA warp.
+// leader's stage barrier (cta_group::2 tensor loads and, gate/up, 4-row
+// tensor gathers of the token rows; no multicast); the leader's commits
+// arrive on the barrier at the same offset in both CTAs.  The gathers move a
+// 128-byte row piece per row where cp.async moves 16 bytes per request: with
+// 16-byte requests the gather's request rate bounded the pair gate/up
+// (measured: 7.2 -> 6.3 ms at T = 16384, d = 7168, E = 896, k = 22).  A
+// single CTA gathers twice the rows per stage, and there tensor gathers were
+// slower than cp.async (the tensor unit also carries the weight tiles).
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
     moe_gemm_pair_kernel(const __grid_constant__ GemmParams p) {
@@ -922,8 +926,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + kMaxTmemBufs;
   uint64_t* drain = tempty + kMaxTmemBufs;
-  uint64_t* gfull = drain + 1;                       // rank 1, gate/up: its own gathers landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gfull + S);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -934,11 +937,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      // leader: both producers' expect-tx arrivals (+ gate/up: its 128 gathering
-      // threads and the forwarded arrival of the second CTA's gathers)
-      mbar_init(full + s, MODE == kModeGateUp ? 2 + kGatherThreads + 1 : 2);
+      // leader: both producers' expect-tx arrivals (+ gate/up: those of both
+      // CTAs' gather warps)
+      mbar_init(full + s, MODE == kModeGateUp ? 2 + 2 * kGatherWarps : 2);
       mbar_init(empty + s, 1);
-      mbar_init(gfull + s, kGatherThreads);
     }
     for (int b = 0; b < kMaxTmemBufs; ++b) {
       mbar_init(tfull + b, 1);
@@ -950,6 +952,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
   }
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < 4; ++i) prefetch_tensormap(&p.mapA[i]);
+    if (MODE == kModeGateUp) prefetch_tensormap(&p.mapX);
     if (MODE == kModeDown)
       for (int i = 0; i < 4; ++i) prefetch_tensormap(&p.mapB[0][i]);
   }
@@ -1050,7 +1053,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
             break;
           }
           tc_fence_after();
-          if (MODE == kModeGateUp) fence_proxy_async_smem();
           const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
           const uint64_t bdesc = sw128_kmajor_desc(sbase + NA * kATileBytes);
           uint64_t adesc[NA];
@@ -1078,34 +1080,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
         tc_commit_pair(drain, 0x1);
         mbar_wait_drain(drain, 0, p.timeout_ns);
       }
-    } else if (lane == 0 && MODE == kModeGateUp) {
-      // ---------------------------------------------------------- rank 1: forward gather completion
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int u = pair; ok && u < num_units; u += npairs) {
-        const int KB = p.d / kTileK;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&gfull[stage], phase, abort_flag, p.err, p.timeout_ns)) {
-            ok = false;
-            break;
-          }
-          fence_proxy_async_smem();
-          mbar_arrive_cluster(full_leader + 8u * stage);
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
     }
     __syncwarp();
   } else if (MODE == kModeGateUp && warp >= 2 + EW) {
     // ------------------------------------------------------------ row gather (this CTA's half)
-    const int g = threadIdx.x - 32 * (2 + EW);
-    const int part = g & 7;
-    const int r0 = g >> 3;
-    uint64_t* land = (rank == 0) ? full : gfull;
+    // Gather warp gw lands rows [32 gw, 32 gw + 32) of this CTA's half of
+    // the token tile with 4-row tensor gathers (one 128-byte row piece each,
+    // swizzled by the map like a tiled load); its lane 0 arms the leader's
+    // stage barrier with their bytes and issues them.
+    const int gw = warp - (2 + EW);
     const uint64_t pol_x = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
@@ -1114,41 +1097,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
       const Unit un = get_unit<MODE>(p, u);
       const bool sh = un.g >= p.E;
       const int half = un.n >> 1;
-      const int nr = (r0 < half) ? (half - r0 + 15) >> 4 : 0;      // rows r0 + 16 i < half
-      const int rbase = un.row0 + static_cast<int>(rank) * half;
-      int tok[8];
+      const int nr = min(max(half - 32 * gw, 0), 32);             // a multiple of 16
+      const int rb = un.row0 + static_cast<int>(rank) * half + 32 * gw;
+      // clamped: a row never reads outside x, even for an invalid routing
+      const int my = (lane < nr) ? min(max(sh ? rb + lane : __ldg(p.perm + rb + lane), 0), p.T - 1) : 0;
+      int tk[32];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = rbase + r0 + 16 * i;
-        tok[i] = (i < nr) ? min(max(sh ? r : __ldg(p.perm + r), 0), p.T - 1) : 0;
-      }
+      for (int j = 0; j < 32; ++j) tk[j] = __shfl_sync(0xffffffffu, my, j);
       const int KB = p.d / kTileK;
       for (int kb = 0; kb < KB; ++kb) {
         int got = 1;
-        if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+        if (lane == 0) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
+            got = 0;
+          } else {
+            const uint32_t fb = full_leader + 8u * stage;
+            mbar_arrive_expect_tx_cluster(fb, static_cast<uint32_t>(nr) * 128u);
+            const uint32_t dst = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + NA * kATileBytes +
+                                 static_cast<uint32_t>(32 * gw) * 128u;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (4 * j < nr)
+                tma_gather4_pair(dst + static_cast<uint32_t>(4 * j) * 128u, &p.mapX, fb, kb * kTileK, tk[4 * j],
+                                 tk[4 * j + 1], tk[4 * j + 2], tk[4 * j + 3], pol_x);
+          }
+        }
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) {
           ok = false;
           break;
         }
-        const uint32_t bbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + NA * kATileBytes;
-        const __nv_bfloat16* src0 = reinterpret_cast<const __nv_bfloat16*>(p.x) + kb * kTileK + part * 8;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (i < nr) {
-            const int r = r0 + 16 * i;
-            cp_async_16(bbase + r * 128 + ((part ^ (r & 7)) << 4), src0 + static_cast<size_t>(tok[i]) * p.d,
-                        pol_x);
-          }
-        }
-        cp_async_mbar_arrive_noinc(&land[stage]);
         if (++stage == S) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
-    cp_async_wait_all();
   } else if (warp >= 2 && warp < 2 + EW) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;

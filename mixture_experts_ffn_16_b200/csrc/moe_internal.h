@@ -126,6 +126,7 @@ struct GemmParams {
   CUtensorMap mapA[4];      // A operands: [0],[1] routed (gate, up | down | router); [2],[3] shared
   CUtensorMap mapB[2][4];   // token-row sources ([0] routed / all tokens, [1] shared), boxes of 16/32/64/128 rows
   CUtensorMap mapO[2];      // expert GEMM outputs ([0] routed rows H_r / Y_r, [1] shared rows), boxes of 32 x 16
+  CUtensorMap mapX;         // gate/up on CTA pairs: x rows for 4-row tensor gathers (box of 64 x 1)
   const int4* units;        // work list (gate/up and down)
   const int* num_units_dev; // its length, on the device
   int num_units_host;       // router: number of units

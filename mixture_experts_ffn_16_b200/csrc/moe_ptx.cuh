@@ -169,6 +169,20 @@ __device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* m
   }
 }
 
+// Tensor gather of four rows r0..r3 (the map's box is 64 elements x 1 row) at
+// column c0 into 4 consecutive 128-byte rows of this CTA's shared memory at
+// `dst`, with the map's swizzle, CTA-pair form: the bytes are counted on the
+// barrier at cluster address `bar_cluster` (the leader's).  No multicast.
+__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                                 int r0, int r1, int r2, int r3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+        "r"(r3), "l"(policy)
+      : "memory");
+}
+
 // 2-D tiled store of a shared-memory box (the map's box, row-major, no
 // swizzle) to coordinates (c0 innermost, c1); completes in this thread's
 // current bulk async-group.
