@@ -394,13 +394,13 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
   const int half_sms = sms / 2;
   const double rows_per_expert = static_cast<double>(T) * k / E;
   q.nmax1 = pick_nmax(rows_per_expert);
-  // Experts of 256+ rows on average: both expert GEMMs run on CTA pairs.
+  // Experts of 96+ rows on average: both expert GEMMs run on CTA pairs.
   // Gate/up: each CTA loads half of every token tile (runs then come in
   // multiples of 32).  Down: each CTA holds one 256-column accumulator
   // instead of two, so tensor memory takes two buffers and a unit's epilogue
-  // overlaps the next unit's MMAs.  Below 256 rows the pair's cross-CTA
-  // handshakes cost more than they save (measured).
-  const int pair_bf16 = (q.nmax1 >= 64 && rows_per_expert >= 256.0) ? 1 : 0;
+  // overlaps the next unit's MMAs.  Measured faster than single CTAs at 128,
+  // 170 and 400 rows per expert; smaller experts keep single CTAs.
+  const int pair_bf16 = (q.nmax1 >= 64 && rows_per_expert >= 96.0) ? 1 : 0;
   // FP8 expert weights: single CTAs, token runs of at most 128 (their
   // accumulators share tensor memory with the widened weight tiles).  The
   // workspace layout is the same for both weight formats.
