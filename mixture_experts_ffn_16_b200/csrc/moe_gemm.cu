@@ -58,7 +58,12 @@ __host__ __device__ constexpr int threads_of(int mode, bool f8 = false) {
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kATileBytes = kTileRows * 128;   // 128 weight rows x 64 bf16
-constexpr int kEpiBytes = 8192;                      // transpose staging of the CTA-pair kernel's epilogue warps
+// Epilogue staging of the CTA-pair kernel, per warp: gate/up: a 1 KB
+// transpose buffer; down: a 16-row transpose buffer with 80-byte rows (64
+// bytes of features + 16 of padding, so the 8 rows of a transposed matrix
+// store hit distinct banks) and the combine weights of the warp's columns.
+__host__ __device__ constexpr int pair_epi_bytes_of(int mode) { return mode == kModeDown ? 16384 : 8192; }
+constexpr int kDownStgRow = 80;
 // Epilogue staging of the single-CTA kernel: 2 KB per warp (router: one fp32
 // transpose buffer; expert GEMMs: two 1 KB slots that alternate, so a slot
 // is refilled while the tensor store of the other is in flight).
@@ -116,6 +121,13 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 }
 
 // v[j] for a run-time j in [0, 8), without indexing the array dynamically.
+// Two floats to a bf16 pair (each rounded to nearest even), the first in
+// the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 __device__ __forceinline__ float pick8(const float (&v)[8], int j) {
   float r = v[0];
 #pragma unroll
@@ -921,6 +933,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
   const int S = p.stages;
   const uint32_t stage_bytes = NA * kATileBytes + static_cast<uint32_t>(nmax / 2) * 128u;
   uint8_t* epi = smem + static_cast<size_t>(S) * stage_bytes;
+  constexpr int kEpiBytes = pair_epi_bytes_of(MODE);
   uint64_t* full = reinterpret_cast<uint64_t*>(epi + kEpiBytes);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
@@ -1144,6 +1157,90 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
       const int sidx = sh ? un.g - p.E : 0;
       const int buf = static_cast<int>(ucount % static_cast<uint32_t>(p.nbuf));
       const uint32_t bpar = (ucount / static_cast<uint32_t>(p.nbuf)) & 1u;
+      const int half = (warp - 2) >> 2;                                   // column blocks half*16 + 32 i
+      if constexpr (MODE == kModeDown) {
+        // Warp (q, half): features 32 q .. + 31 of this CTA's 128 rows, token
+        // columns 16 half + 32 i .. + 15 (i < 8).  Each 16-column block is
+        // read from tensor memory as two 16-lane fragments, scaled by the
+        // combine weights in fp32, packed to bf16 pairs and written
+        // transposed (token rows, 64 bytes of features each) by stmatrix,
+        // then stored to global memory as 16-byte row pieces.  The weights
+        // sit in shared memory in block order: wsm[16 i + j] = weight of
+        // column 16 half + 32 i + j.
+        float* wsm = reinterpret_cast<float*>(stg + 16 * kDownStgRow);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int idx = 32 * j + lane;
+          const int c = 16 * half + 32 * (idx >> 4) + (idx & 15);
+          wsm[idx] = (!sh && c < un.n) ? __ldg(p.roww + un.row0 + c) : 1.0f;
+        }
+        __syncwarp();
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&tfull[buf], bpar, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) break;
+        tc_fence_after();
+        const uint32_t tbase =
+            tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * nmax);
+        const int feat0 = un.wb * kWbRows + static_cast<int>(rank) * kTileRows + 32 * q;
+        if (feat0 < p.d) {
+          __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(sh ? p.out_s : p.out_r);
+          const size_t rbase = (sh ? static_cast<size_t>(sidx) * p.Tp : 0) + static_cast<size_t>(un.row0);
+          const uint32_t sbase = smem_u32(stg);
+          const int tq = lane & 3;
+          const int mi = lane >> 3, mj = lane & 7;     // this thread's stmatrix row: matrix mi, row mj
+          uint32_t va[2][8], vb[2][8];
+          auto load = [&](uint32_t (&v)[2][8], int c) {
+            tmem_ld_16x256b_x2(tbase + static_cast<uint32_t>(c), v[0]);
+            tmem_ld_16x256b_x2(tbase + (16u << 16) + static_cast<uint32_t>(c), v[1]);
+          };
+          auto emit = [&](const uint32_t (&v)[2][8], int i) {
+            const int c = 16 * half + 32 * i;
+            const float2 w0 = *reinterpret_cast<const float2*>(wsm + 16 * i + 2 * tq);
+            const float2 w1 = *reinterpret_cast<const float2*>(wsm + 16 * i + 8 + 2 * tq);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              // matrices: 0 = features 16h + 0..7 x tokens 0..7, 1 = features
+              // 16h + 8..15 x tokens 0..7, 2 and 3 = the same for tokens 8..15
+              const uint32_t m0 = pack_bf16x2(__uint_as_float(v[h][0]) * w0.x, __uint_as_float(v[h][1]) * w0.y);
+              const uint32_t m1 = pack_bf16x2(__uint_as_float(v[h][2]) * w0.x, __uint_as_float(v[h][3]) * w0.y);
+              const uint32_t m2 = pack_bf16x2(__uint_as_float(v[h][4]) * w1.x, __uint_as_float(v[h][5]) * w1.y);
+              const uint32_t m3 = pack_bf16x2(__uint_as_float(v[h][6]) * w1.x, __uint_as_float(v[h][7]) * w1.y);
+              stmatrix_x4_trans(sbase + static_cast<uint32_t>((8 * (mi >> 1) + mj) * kDownStgRow +
+                                                              (16 * h + 8 * (mi & 1)) * 2),
+                                m0, m1, m2, m3);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int rep = 0; rep < 2; ++rep) {
+              const int cc = lane + 32 * rep;
+              const int tok = cc >> 2, part = cc & 3;
+              const uint4 o = *reinterpret_cast<const uint4*>(stg + tok * kDownStgRow + part * 16);
+              *reinterpret_cast<uint4*>(outp + (rbase + c + tok) * p.d + feat0 + part * 8) = o;
+            }
+            __syncwarp();
+          };
+          // two fragment sets: the next block's loads are in flight while the
+          // current one is converted and stored
+          if (16 * half < un.n) load(va, 16 * half);
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            if (16 * half + 32 * i >= un.n) break;
+            tmem_ld_wait();
+            if (16 * half + 32 * (i + 1) < un.n) load(vb, 16 * half + 32 * (i + 1));
+            emit(va, i);
+            if (16 * half + 32 * (i + 1) >= un.n) break;
+            tmem_ld_wait();
+            if (i + 2 < 8 && 16 * half + 32 * (i + 2) < un.n) load(va, 16 * half + 32 * (i + 2));
+            emit(vb, i + 1);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_leader + 8u * buf);
+        ++ucount;
+        continue;
+      }
       // down: combine weights of the unit's rows, fetched before the wait
       // (lane l of register j holds the weight of column 32 j + l)
       float wreg[8];
@@ -1157,7 +1254,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) break;
       tc_fence_after();
-      const int half = (warp - 2) >> 2;                                   // column blocks half*16 + 32 i
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * NA * nmax);
       const int feat0 = un.wb * kWbRows + static_cast<int>(rank) * kTileRows + 32 * q;
@@ -1250,7 +1346,7 @@ size_t gemm_smem_bytes(int mode, int nmax, int* stages) {
 size_t gemm_pair_smem_bytes(int mode, int nmax, int* stages) {
   const int NA = (mode == kModeGateUp) ? 2 : 1;
   const size_t stage_bytes = NA * static_cast<size_t>(kATileBytes) + static_cast<size_t>(nmax / 2) * 128;
-  const size_t fixed = kSmemAlign + kEpiBytes + kSmemTail;
+  const size_t fixed = kSmemAlign + pair_epi_bytes_of(mode) + kSmemTail;
   const size_t budget = 232448;
   int s = static_cast<int>((budget - fixed) / stage_bytes);
   if (s > kMaxStages) s = kMaxStages;

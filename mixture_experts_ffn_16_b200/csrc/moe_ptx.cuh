@@ -388,6 +388,28 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
+// One load of 16 lanes x 16 columns (shape 16x256b, repeated twice along the
+// columns).  Thread t receives lane t/4 at columns 2 (t%4) and 2 (t%4) + 1
+// (r[0], r[1]), lane 8 + t/4 at the same columns (r[2], r[3]), and the same
+// four for the columns 8 further on (r[4..7]): the register layout of an
+// 8 x 8 matrix fragment, as stmatrix takes it.
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+// Four 8 x 8 matrices of 16-bit values from registers (register i of thread t
+// holds row t/4, columns 2 (t%4) and 2 (t%4) + 1 of matrix i, the lower
+// column in the low half), stored transposed: column j of matrix i goes to
+// the 16 bytes at the shared-memory address that thread 8 i + j passes.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                                  uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(r0),
+               "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
