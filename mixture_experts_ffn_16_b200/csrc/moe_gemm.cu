@@ -58,12 +58,12 @@ __host__ __device__ constexpr int threads_of(int mode, bool f8 = false) {
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kATileBytes = kTileRows * 128;   // 128 weight rows x 64 bf16
-// Epilogue staging of the CTA-pair kernel, per warp: gate/up: a 1 KB
-// transpose buffer; down: a 16-row transpose buffer with 80-byte rows (64
-// bytes of features + 16 of padding, so the 8 rows of a transposed matrix
-// store hit distinct banks) and the combine weights of the warp's columns.
-__host__ __device__ constexpr int pair_epi_bytes_of(int mode) { return mode == kModeDown ? 16384 : 8192; }
-constexpr int kDownStgRow = 80;
+// Epilogue staging of the CTA-pair kernel: 2 KB per warp, a 16-row transpose
+// buffer with 80-byte rows (64 bytes of features + 16 of padding, so the 8
+// rows of a transposed matrix store hit distinct banks) and, down, the
+// combine weights of the warp's columns.
+__host__ __device__ constexpr int pair_epi_bytes_of(int) { return 16384; }
+constexpr int kStgRow = 80;
 // Epilogue staging of the single-CTA kernel: 2 KB per warp (router: one fp32
 // transpose buffer; expert GEMMs: two 1 KB slots that alternate, so a slot
 // is refilled while the tensor store of the other is in flight).
@@ -1167,7 +1167,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
         // then stored to global memory as 16-byte row pieces.  The weights
         // sit in shared memory in block order: wsm[16 i + j] = weight of
         // column 16 half + 32 i + j.
-        float* wsm = reinterpret_cast<float*>(stg + 16 * kDownStgRow);
+        float* wsm = reinterpret_cast<float*>(stg + 16 * kStgRow);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int idx = 32 * j + lane;
@@ -1206,7 +1206,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
               const uint32_t m1 = pack_bf16x2(__uint_as_float(v[h][2]) * w0.x, __uint_as_float(v[h][3]) * w0.y);
               const uint32_t m2 = pack_bf16x2(__uint_as_float(v[h][4]) * w1.x, __uint_as_float(v[h][5]) * w1.y);
               const uint32_t m3 = pack_bf16x2(__uint_as_float(v[h][6]) * w1.x, __uint_as_float(v[h][7]) * w1.y);
-              stmatrix_x4_trans(sbase + static_cast<uint32_t>((8 * (mi >> 1) + mj) * kDownStgRow +
+              stmatrix_x4_trans(sbase + static_cast<uint32_t>((8 * (mi >> 1) + mj) * kStgRow +
                                                               (16 * h + 8 * (mi & 1)) * 2),
                                 m0, m1, m2, m3);
             }
@@ -1215,7 +1215,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
             for (int rep = 0; rep < 2; ++rep) {
               const int cc = lane + 32 * rep;
               const int tok = cc >> 2, part = cc & 3;
-              const uint4 o = *reinterpret_cast<const uint4*>(stg + tok * kDownStgRow + part * 16);
+              const uint4 o = *reinterpret_cast<const uint4*>(stg + tok * kStgRow + part * 16);
               *reinterpret_cast<uint4*>(outp + (rbase + c + tok) * p.d + feat0 + part * 8) = o;
             }
             __syncwarp();
@@ -1241,14 +1241,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
         ++ucount;
         continue;
       }
-      // down: combine weights of the unit's rows, fetched before the wait
-      // (lane l of register j holds the weight of column 32 j + l)
-      float wreg[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = 32 * j + lane;
-        wreg[j] = (MODE == kModeDown && !sh && c < un.n) ? __ldg(p.roww + un.row0 + c) : 1.0f;
-      }
+      // gate/up: H = SiLU(gate) * up for features 32 q .. + 31 of this CTA's
+      // 128 rows and the same token columns as down, through the same
+      // fragment loads and transposed stmatrix stores.
       int got = 1;
       if (lane == 0) got = mbar_wait(&tfull[buf], bpar, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
       got = __shfl_sync(0xffffffffu, got, 0);
@@ -1257,61 +1252,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * NA * nmax);
       const int feat0 = un.wb * kWbRows + static_cast<int>(rank) * kTileRows + 32 * q;
-      const int wrows = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
-      if (feat0 < wrows) {
-        const int ld = (MODE == kModeGateUp) ? (sh ? p.fs : p.f) : p.d;
+      const int ld = sh ? p.fs : p.f;
+      if (feat0 < ld) {
         __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(sh ? p.out_s : p.out_r);
         const size_t rbase = (sh ? static_cast<size_t>(sidx) * p.Tp : 0) + static_cast<size_t>(un.row0);
-        auto emit = [&](const uint32_t (&A)[16], const uint32_t (&B)[16], int c, float wsel) {
-          __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
-          if (MODE == kModeGateUp) {
+        const uint32_t sbase = smem_u32(stg);
+        const int mi = lane >> 3, mj = lane & 7;
+        uint32_t ga[2][8], ua[2][8], gb[2][8], ub[2][8];
+        auto load = [&](uint32_t (&g)[2][8], uint32_t (&v)[2][8], int c) {
+          tmem_ld_16x256b_x2(tbase + static_cast<uint32_t>(c), g[0]);
+          tmem_ld_16x256b_x2(tbase + (16u << 16) + static_cast<uint32_t>(c), g[1]);
+          tmem_ld_16x256b_x2(tbase + static_cast<uint32_t>(nmax + c), v[0]);
+          tmem_ld_16x256b_x2(tbase + (16u << 16) + static_cast<uint32_t>(nmax + c), v[1]);
+        };
+        auto emit = [&](const uint32_t (&g)[2][8], const uint32_t (&v)[2][8], int i) {
+          const int c = 16 * half + 32 * i;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float gg = __uint_as_float(A[i]);
-              const float vv = __uint_as_float(B[i]);
-              sb[i * 32 + lane] = __float2bfloat16_rn(silu_f(gg) * vv);
-            }
-          } else {
+          for (int h = 0; h < 2; ++h) {
+            uint32_t m[4];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float w = __shfl_sync(0xffffffffu, wsel, (c + i) & 31);
-              sb[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(A[i]) * w);
-            }
+            for (int k = 0; k < 4; ++k)
+              m[k] = pack_bf16x2(silu_f(__uint_as_float(g[h][2 * k])) * __uint_as_float(v[h][2 * k]),
+                                 silu_f(__uint_as_float(g[h][2 * k + 1])) * __uint_as_float(v[h][2 * k + 1]));
+            stmatrix_x4_trans(
+                sbase + static_cast<uint32_t>((8 * (mi >> 1) + mj) * kStgRow + (16 * h + 8 * (mi & 1)) * 2), m[0],
+                m[1], m[2], m[3]);
           }
           __syncwarp();
 #pragma unroll
           for (int rep = 0; rep < 2; ++rep) {
             const int cc = lane + 32 * rep;
             const int tok = cc >> 2, part = cc & 3;
-            const uint4 v = *reinterpret_cast<const uint4*>(stg + tok * 64 + part * 16);
-            *reinterpret_cast<uint4*>(outp + (rbase + c + tok) * ld + feat0 + part * 8) = v;
+            const uint4 o = *reinterpret_cast<const uint4*>(stg + tok * kStgRow + part * 16);
+            *reinterpret_cast<uint4*>(outp + (rbase + c + tok) * ld + feat0 + part * 8) = o;
           }
           __syncwarp();
         };
-        constexpr int kStep = 32;
-        uint32_t a0[16], b0[16], a1[16], b1[16];
-        int c0 = 16 * half;
-        if (c0 < un.n) {
-          tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c0), a0);
-          if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c0), b0);
-        }
-        while (c0 < un.n) {
+        if (16 * half < un.n) load(ga, ua, 16 * half);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          if (16 * half + 32 * i >= un.n) break;
           tmem_ld_wait();
-          const int c1 = c0 + kStep;
-          if (c1 < un.n) {
-            tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c1), a1);
-            if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c1), b1);
-          }
-          emit(a0, b0, c0, MODE == kModeDown ? pick8(wreg, c0 >> 5) : 1.0f);
-          if (c1 >= un.n) break;
+          if (16 * half + 32 * (i + 1) < un.n) load(gb, ub, 16 * half + 32 * (i + 1));
+          emit(ga, ua, i);
+          if (16 * half + 32 * (i + 1) >= un.n) break;
           tmem_ld_wait();
-          const int c2 = c1 + kStep;
-          if (c2 < un.n) {
-            tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(c2), a0);
-            if (MODE == kModeGateUp) tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(nmax + c2), b0);
-          }
-          emit(a1, b1, c1, MODE == kModeDown ? pick8(wreg, c1 >> 5) : 1.0f);
-          c0 = c2;
+          if (i + 2 < 8 && 16 * half + 32 * (i + 2) < un.n) load(ga, ua, 16 * half + 32 * (i + 2));
+          emit(gb, ub, i + 1);
         }
       }
       tc_fence_before();
