@@ -213,7 +213,16 @@ __device__ __forceinline__ void widen_block(const uint4 v0, const uint4 v1, uint
 
 // SiLU(z) = z * sigmoid(z) with the fast exponential and division; the
 // exponent is clamped so the denominator stays finite (|result| < 1e-32 there).
-__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(fminf(-z, 80.0f))); }
+// SiLU(z) = z * sigmoid(z), with sigmoid(z) = (1 + tanh(z / 2)) / 2: one
+// special-function op (tanh.approx, relative error about 2^-11, below the
+// bf16 rounding of the result) where exp and a reciprocal take two; the
+// special-function unit's rate bounds the gate/up epilogue.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float silu_f(float z) { return z * fmaf(0.5f, tanh_approx(0.5f * z), 0.5f); }
 
 // F8: the routed and shared expert weights are block-scaled FP8 (codes plus
 // one power-of-two scale per 32 codes along K).  The producer lands code and
