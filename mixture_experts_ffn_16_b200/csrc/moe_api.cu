@@ -151,10 +151,10 @@ cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s
 
 // ---- the steps, after validation ----
 
-int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_router, const float* bias,
-              int score_fn, int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w, char* ws,
-              cudaStream_t st) {
-  if (cudaMemsetAsync(ws + p.err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+// The router GEMM of plan p: partial logits [router_split, T, E] fp32 at
+// `logits`, on single CTAs or CTA pairs as the plan chose.
+int launch_router_gemm(const Plan& p, const DeviceInfo& di, const void* x, const void* W_router, float* logits,
+                       uint32_t* err, cudaStream_t st) {
   GemmParams g;
   std::memset(&g, 0, sizeof g);
   if (!map_weights(&g.mapA[0], W_router, p.d, p.E, 1) || !map_rows_set(g.mapB[0], x, p.d, p.T))
@@ -162,23 +162,38 @@ int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_
   g.mapA[1] = g.mapA[2] = g.mapA[3] = g.mapA[0];
   copy_set(g.mapB[1], g.mapB[0]);
   g.num_units_host = p.router_units;
-  g.out_r = ws + p.logits;
-  g.err = reinterpret_cast<uint32_t*>(ws + p.err);
-  g.T = p.T; g.Tp = p.Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
+  g.out_r = logits;
+  g.err = err;
+  g.T = p.T; g.Tp = p.router_Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
   g.nmax = p.nmax_r;
-  g.router_nwb = p.nwbE;
+  g.router_nwb = p.router_nwb;
   g.router_split = p.router_split;
   g.router_kbs = p.router_kbs;
   g.timeout_ns = kWaitTimeoutNs;
+  g.nbuf = 512 / p.nmax_r < 8 ? 512 / p.nmax_r : 8;   // partial-logit buffers drained in turn
   int stages = 0;
+  if (p.router_pair) {
+    const size_t smem = gemm_pair_smem_bytes(kModeRouter, p.nmax_r, &stages);
+    g.stages = stages;
+    const int grid = 2 * p.router_units < di.sms ? 2 * p.router_units : di.sms;
+    return launch_gemm_pair(kModeRouter, g, grid, smem, st);
+  }
   const size_t smem = gemm_smem_bytes(kModeRouter, p.nmax_r, &stages);
   g.stages = stages;
-  g.nbuf = 512 / p.nmax_r < 8 ? 512 / p.nmax_r : 8;   // partial-logit buffers drained in turn
   const int grid = p.router_units < di.sms ? p.router_units : di.sms;
-  int rc = launch_gemm(kModeRouter, g, grid, smem, st);
+  return launch_gemm(kModeRouter, g, grid, smem, st);
+}
+
+int run_route(const Plan& p, const DeviceInfo& di, const void* x, const void* W_router, const float* bias,
+              int score_fn, int norm_topk, float route_scale, int32_t* topk_idx, float* topk_w, char* ws,
+              cudaStream_t st) {
+  if (cudaMemsetAsync(ws + p.err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+  float* logits = reinterpret_cast<float*>(ws + p.logits);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws + p.err);
+  const int rc = launch_router_gemm(p, di, x, W_router, logits, err, st);
   if (rc != MOE_OK) return rc;
-  return launch_topk(reinterpret_cast<const float*>(ws + p.logits), p.router_split, bias, p.T, p.E, p.k, score_fn,
-                     norm_topk, route_scale, topk_idx, topk_w, g.err, st);
+  return launch_topk(logits, p.router_split, bias, p.T, p.E, p.k, score_fn, norm_topk, route_scale, topk_idx,
+                     topk_w, err, st);
 }
 
 int run_gate_up(const Plan& p, const DeviceInfo& di, const void* x, Wt Wg, Wt Wu, Wt Wsg, Wt Wsu, char* ws,
@@ -425,6 +440,7 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
   // registers) when that still gives every SM a unit; else runs of 64 or
   // narrower while most SMs stay busy.
   q.nmax_r = 16;
+  q.router_pair = 0;
   if (static_cast<long long>(q.nwbE) * ceil_div(q.Tp, 128) >= sms) {
     q.nmax_r = 128;
   } else {
@@ -440,6 +456,7 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
   {
     const int base = q.nwbE * ceil_div(q.Tp, q.nmax_r);
     const int KB = d / kTileK;
+    const int Tp32 = ceil_div(T, 2 * kRowPad) * 2 * kRowPad;
     int split = 1;
     if (base < half_sms) {
       split = sms / base;
@@ -448,36 +465,45 @@ int make_plan(const moe_shape* s, Plan* p, bool f8) {
       if (split < 1) split = 1;
     } else {
       // Enough runs for most SMs: the launch is bound by what each SM must
-      // load, (units per SM) x (128 + n) rows x its K slice.  Wider runs
-      // re-read W_router less; a second K slice spreads the runs over more
+      // load, (units per SM) x (128 + its token rows) x its K slice.  Wider
+      // runs re-read W_router less; a CTA pair (256 experts x 256 tokens per
+      // unit, each CTA loading 128 of each) halves the bytes per logit
+      // again (pairs with 128-token runs measured slower than single CTAs
+      // on prefill_softmax); a second K slice spreads the units over more
       // SMs but adds a partial-logit array, written here and read back by
       // top-k.  Another tiling replaces the rule above only when this model
       // calls it clearly cheaper (measured: prefill_softmax routing
       // 32.5 -> 26.4 us with 128-token runs in two slices).
-      auto cost = [&](int n, int sp) {
+      auto cost = [&](int pr, int n, int sp) {
         const int kbs = ceil_div(KB, sp);
         const int ns = ceil_div(KB, kbs);
-        const long long units = static_cast<long long>(q.nwbE) * ceil_div(q.Tp, n) * ns;
-        const long long per_sm = (units + sms - 1) / sms;
-        const double ingest = static_cast<double>(per_sm) * (kTileRows + n) * kbs * kTileK * 2;
+        const int slots = pr ? half_sms : sms;
+        const long long units = static_cast<long long>(ceil_div(E, pr ? 2 * kTileRows : kTileRows)) *
+                                ceil_div(pr ? Tp32 : q.Tp, n) * ns;
+        const long long per = (units + slots - 1) / slots;
+        const double ingest = static_cast<double>(per) * (kTileRows + (pr ? n / 2 : n)) * kbs * kTileK * 2;
         const double partials = static_cast<double>(ns - 1) * T * E * 4 * 2;
         return ingest / 47e9 + partials / 6.5e12;
       };
-      const double c0 = cost(q.nmax_r, 1);
+      const double c0 = cost(0, q.nmax_r, 1);
       double best = 0.9 * c0;
       int bn = q.nmax_r;
-      for (int n = 32; n <= 128; n <<= 1)
-        for (int sp = 1; sp <= 2 && sp <= KB; ++sp) {
-          const double c = cost(n, sp);
-          if (c < best) {
-            best = c;
-            bn = n;
-            split = sp;
+      for (int pr = 0; pr <= 1; ++pr)
+        for (int n = pr ? 256 : 32; n <= (pr ? 256 : 128); n <<= 1)
+          for (int sp = 1; sp <= 2 && sp <= KB; ++sp) {
+            const double c = cost(pr, n, sp);
+            if (c < best) {
+              best = c;
+              bn = n;
+              split = sp;
+              q.router_pair = pr;
+            }
           }
-        }
       q.nmax_r = bn;
     }
-    const int runs = q.nwbE * ceil_div(q.Tp, q.nmax_r);
+    q.router_nwb = q.router_pair ? ceil_div(E, 2 * kTileRows) : q.nwbE;
+    q.router_Tp = q.router_pair ? Tp32 : q.Tp;
+    const int runs = q.router_nwb * ceil_div(q.router_Tp, q.nmax_r);
     q.router_kbs = ceil_div(KB, split);
     q.router_split = ceil_div(KB, q.router_kbs);   // no empty slice
     q.router_units = runs * q.router_split;
@@ -964,27 +990,7 @@ extern "C" int moe_route_noalloc(const moe_shape* shape, const void* x, const vo
   float* logits = reinterpret_cast<float*>(scratch + kNoAllocHeaderBytes);
   // The array keeps the previous call's contents: the error word must start at zero.
   if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
-  GemmParams g;
-  std::memset(&g, 0, sizeof g);
-  if (!map_weights(&g.mapA[0], W_router, p.d, p.E, 1) || !map_rows_set(g.mapB[0], x, p.d, p.T))
-    return MOE_ERR_CUDA;
-  g.mapA[1] = g.mapA[2] = g.mapA[3] = g.mapA[0];
-  copy_set(g.mapB[1], g.mapB[0]);
-  g.num_units_host = p.router_units;
-  g.out_r = logits;
-  g.err = err;
-  g.T = p.T; g.Tp = p.Tp; g.E = p.E; g.d = p.d; g.f = p.f; g.fs = p.fs;
-  g.nmax = p.nmax_r;
-  g.router_nwb = p.nwbE;
-  g.router_split = p.router_split;
-  g.router_kbs = p.router_kbs;
-  g.timeout_ns = kWaitTimeoutNs;
-  int stages = 0;
-  const size_t smem = gemm_smem_bytes(kModeRouter, p.nmax_r, &stages);
-  g.stages = stages;
-  g.nbuf = 512 / p.nmax_r < 8 ? 512 / p.nmax_r : 8;
-  const int grid = p.router_units < di.sms ? p.router_units : di.sms;
-  if ((rc = launch_gemm(kModeRouter, g, grid, smem, st)) != MOE_OK) return rc;
+  if ((rc = launch_router_gemm(p, di, x, W_router, logits, err, st)) != MOE_OK) return rc;
   return launch_topk(logits, p.router_split, expert_bias, p.T, p.E, p.k, score_fn, norm_topk, route_scale, topk_idx,
                      topk_w, err, st);
 }

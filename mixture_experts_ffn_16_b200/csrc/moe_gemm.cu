@@ -9,7 +9,8 @@
 // consecutive rows of the group's row segment); for the router, g is a slice
 // of d instead when the plan splits K, each slice writing its own partial
 // logits.  A CTA-pair form (cta_group::2, moe_gemm_pair_kernel) serves the
-// gate/up GEMM of large experts.  The GEMM is "swap-AB": the
+// expert GEMMs of large experts and the router of large batches (256
+// experts x 256 tokens per unit).  The GEMM is "swap-AB": the
 // 128 weight rows are the MMA's M side and the unit's tokens its N side
 // (n a multiple of 16), so an expert with few tokens costs n/16 MMA columns,
 // not a padded 128-row tile.
@@ -20,9 +21,10 @@
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer; fp32
 //               accumulators in tensor memory (gate and up side by side for
 //               the gate/up GEMM), double-buffered when they fit.
-//   epilogue    4 (router) or 8 warps: tcgen05.ld -> fp32 math (SiLU*, weight
-//               scale) -> bf16 -> transpose through shared memory -> 16-byte
-//               stores of whole row segments.
+//   epilogue    4 (router; 8 in its pair form) or 8 warps: tcgen05.ld ->
+//               fp32 math (SiLU*, weight scale; router: fp32 sums of the
+//               drained partial logits) -> bf16 -> transpose through shared
+//               memory -> 16-byte stores of whole row segments.
 //   gather      gate/up: 4 warps copy the unit's token rows of x (by perm)
 //               straight into the swizzled tile (cp.async; CTA pairs: 4-row
 //               tensor gathers); no permuted copy of x is ever made.
@@ -58,6 +60,14 @@ __host__ __device__ constexpr int threads_of(int mode, bool f8 = false) {
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kATileBytes = kTileRows * 128;   // 128 weight rows x 64 bf16
+// CTA-pair kernel: 8 epilogue warps in every mode (router: two per tensor-
+// memory lane quarter, each summing half of the run's token columns).
+__host__ __device__ constexpr int pair_epi_warps_of(int) { return 8; }
+// Token rows: gate/up gathers them with kGatherWarps warps; down and the
+// router load them with tiled tensor loads from a second producer warp.
+__host__ __device__ constexpr int pair_threads_of(int mode) {
+  return 64 + 32 * pair_epi_warps_of(mode) + (mode == kModeGateUp ? kGatherThreads : 32);
+}
 // Epilogue staging of the CTA-pair kernel: 2 KB per warp, a 16-row transpose
 // buffer with 80-byte rows (64 bytes of features + 16 of padding, so the 8
 // rows of a transposed matrix store hit distinct banks) and, down, the
@@ -211,12 +221,14 @@ __device__ __forceinline__ void widen_block(const uint4 v0, const uint4 v1, uint
   o[12] = d.x; o[13] = d.y; o[14] = d.z; o[15] = d.w;
 }
 
-// SiLU(z) = z * sigmoid(z) with the fast exponential and division; the
-// exponent is clamped so the denominator stays finite (|result| < 1e-32 there).
 // SiLU(z) = z * sigmoid(z), with sigmoid(z) = (1 + tanh(z / 2)) / 2: one
-// special-function op (tanh.approx, relative error about 2^-11, below the
-// bf16 rounding of the result) where exp and a reciprocal take two; the
-// special-function unit's rate bounds the gate/up epilogue.
+// special-function op (tanh.approx) where exp and a reciprocal take two; the
+// special-function unit's rate bounds the gate/up epilogue.  tanh.approx has a
+// relative error of about 2^-11, so sigmoid's absolute error is at most about
+// 2^-12: for z >= 0 that is below the bf16 rounding of h, while for z << 0
+// (sigmoid near 0) SiLU's absolute error, about |z| * 2^-12, can exceed the
+// relative bf16 rounding of that small value; it stays far inside the
+// block's output tolerance (max |err| <= 2e-2 * max |out|).
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -918,6 +930,13 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
 //   down    : wb = 256-row block of d; A tile per CTA: its 128 rows (one
 //             256-column accumulator per CTA, so tensor memory holds two
 //             buffers and the epilogue of one unit overlaps the next's MMAs).
+//   router  : wb = 256-expert block of E, g = the unit's slice of d; A tile
+//             per CTA: its 128 rows of W_router, B its half of the run's
+//             token rows of x.  Each CTA thus loads 128 + 128 rows per k-block
+//             for 128 x 256 logits where a single CTA loads 128 + 128 for
+//             128 x 128.  The accumulator is drained every kRouterDrainKB
+//             k-blocks through two buffers of 256 columns by 8 epilogue warps
+//             (128 fp32 sums each).
 // The leader CTA (rank 0) issues the MMAs; loads of both CTAs complete on the
 // leader's stage barrier (cta_group::2 tensor loads and, gate/up, 4-row
 // tensor gathers of the token rows; no multicast); the leader's commits
@@ -928,12 +947,12 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
 // single CTA gathers twice the rows per stage, and there tensor gathers were
 // slower than cp.async (the tensor unit also carries the weight tiles).
 template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE), 1)
     moe_gemm_pair_kernel(const __grid_constant__ GemmParams p) {
-  static_assert(MODE == kModeGateUp || MODE == kModeDown, "pair kernel serves the expert GEMMs");
-  // gate/up: gate and up tile of this CTA's 128 rows; down: one 128-row tile.
+  // gate/up: gate and up tile of this CTA's 128 rows; down and router: one
+  // 128-row tile.
   constexpr int NA = (MODE == kModeGateUp) ? 2 : 1;
-  constexpr int EW = epi_warps_of(MODE);
+  constexpr int EW = pair_epi_warps_of(MODE);
   constexpr int kWbRows = 2 * kTileRows;   // weight rows per pair-unit (128 per CTA)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -959,9 +978,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      // leader: both producers' expect-tx arrivals (+ gate/up: those of both
-      // CTAs' gather warps)
-      mbar_init(full + s, MODE == kModeGateUp ? 2 + 2 * kGatherWarps : 2);
+      // leader: the weight producers' expect-tx arrivals of both CTAs, plus
+      // those of both CTAs' gather warps (gate/up) or token producers
+      mbar_init(full + s, MODE == kModeGateUp ? 2 + 2 * kGatherWarps : 4);
       mbar_init(empty + s, 1);
     }
     for (int b = 0; b < kMaxTmemBufs; ++b) {
@@ -975,7 +994,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < 4; ++i) prefetch_tensormap(&p.mapA[i]);
     if (MODE == kModeGateUp) prefetch_tensormap(&p.mapX);
-    if (MODE == kModeDown)
+    if (MODE != kModeGateUp)
       for (int i = 0; i < 4; ++i) prefetch_tensormap(&p.mapB[0][i]);
   }
   if (warp == 1) {
@@ -988,8 +1007,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   chain_wait();
-  int num_units = *p.num_units_dev;
-  if (*p.plan_tag_dev != p.plan_tag) {
+  int num_units = (MODE == kModeRouter) ? p.num_units_host : *p.num_units_dev;
+  if (MODE != kModeRouter && *p.plan_tag_dev != p.plan_tag) {
     if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(p.err, kDevErrPlanMismatch);
     num_units = 0;
   }
@@ -997,28 +1016,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
   const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0); // + 8 * buf
 
   if (warp == 0) {
-    // ------------------------------------------------------------ weight (and down: token) loads
-    const uint64_t pol_a = p.weights_evict_first ? policy_evict_first() : policy_evict_last();
-    const uint64_t pol_b = policy_evict_last();
+    // ------------------------------------------------------------ weight loads
+    // router: W_router is re-read by every token run -> keep
+    const uint64_t pol_a =
+        (MODE != kModeRouter && p.weights_evict_first) ? policy_evict_first() : policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued = 0;
     bool ok = true;
     for (int u = pair; ok && u < num_units; u += npairs) {
       const Unit un = get_unit<MODE>(p, u);
-      const bool sh = un.g >= p.E;
+      const bool sh = (MODE != kModeRouter) && un.g >= p.E;
       const int sidx = sh ? un.g - p.E : 0;
       const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
       const int KB = K / kTileK;
+      // router: this unit's k-blocks [kb0, kb1) (its slice of d); the expert GEMMs: all of K
+      const int kb0 = (MODE == kModeRouter) ? un.g * p.router_kbs : 0;
+      const int kb1 = (MODE == kModeRouter) ? min(KB, kb0 + p.router_kbs) : KB;
       const CUtensorMap* mA = &p.mapA[sh ? 2 : 0];
-      const CUtensorMap* mB = p.mapB[sh ? 1 : 0];
-      const int a_c2 = sh ? sidx : un.g;
-      const int half = un.n >> 1;
-      const int brow0 = (sh ? sidx * p.Tp : 0) + un.row0 + static_cast<int>(rank) * half;
-      const uint32_t tx_bytes = NA * kATileBytes + (MODE == kModeDown ? static_cast<uint32_t>(half) * 128u : 0u);
+      const int a_c2 = (MODE == kModeRouter) ? 0 : (sh ? sidx : un.g);
+      const uint32_t tx_bytes = NA * kATileBytes;
       int got = 1;
       if (lane == 0) {
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
             got = 0;
             break;
@@ -1030,8 +1050,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
           for (int a = 0; a < NA; ++a)
             tma_load_3d_pair_hint(sbase + a * kATileBytes, mA + a, fb, kb * kTileK,
                                   un.wb * kWbRows + static_cast<int>(rank) * kTileRows, a_c2, pol_a);
-          if (MODE == kModeDown)
-            tma_load_rows<true>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, half, pol_b);
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -1058,7 +1076,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
       uint32_t ucount = 0;
       bool any = false;
       bool ok = true;
-      for (int u = pair; ok && u < num_units; u += npairs) {
+      if constexpr (MODE == kModeRouter) {
+        // Router: M = 256 experts (128 per CTA), N = the run's tokens; the
+        // accumulator is drained every kRouterDrainKB k-blocks into fp32
+        // registers by both CTAs' epilogues (as in the single-CTA router),
+        // through nbuf buffers of nmax columns.
+        uint32_t dc = 0;
+        for (int u = pair; ok && u < num_units; u += npairs) {
+          const Unit un = get_unit<MODE>(p, u);
+          const int KB = p.d / kTileK;
+          const int kb0 = un.g * p.router_kbs;
+          const int kb1 = min(KB, kb0 + p.router_kbs);
+          const uint32_t idesc = idesc_bf16_f32(2 * kTileRows, un.n);
+          uint32_t dcol = tmem_base;
+          int buf = 0;
+          for (int kb = kb0; kb < kb1; ++kb) {
+            const int sub = (kb - kb0) % kRouterDrainKB;
+            if (sub == 0) {
+              buf = static_cast<int>(dc % static_cast<uint32_t>(p.nbuf));
+              const uint32_t bpar = (dc / static_cast<uint32_t>(p.nbuf)) & 1u;
+              if (!mbar_wait(&tempty[buf], bpar ^ 1u, abort_flag, p.err, p.timeout_ns)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              dcol = tmem_base + static_cast<uint32_t>(buf * nmax);
+            }
+            if (!mbar_wait(&full[stage], phase, abort_flag, p.err, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+            const uint64_t adesc = sw128_kmajor_desc(sbase);
+            const uint64_t bdesc = sw128_kmajor_desc(sbase + kATileBytes);
+#pragma unroll
+            for (int ks = 0; ks < kTileK / 16; ++ks)
+              tc_mma_bf16_pair(dcol, adesc + 2u * ks, bdesc + 2u * ks, idesc, (sub | ks) != 0 ? 1u : 0u);
+            any = true;
+            tc_commit_pair(&empty[stage], 0x3);
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            if (sub == kRouterDrainKB - 1 || kb == kb1 - 1) {
+              tc_commit_pair(&tfull[buf], 0x3);
+              ++dc;
+            }
+          }
+        }
+      }
+      for (int u = pair; MODE != kModeRouter && ok && u < num_units; u += npairs) {
         const Unit un = get_unit<MODE>(p, u);
         const bool sh = un.g >= p.E;
         const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
@@ -1104,6 +1172,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
       }
     }
     __syncwarp();
+  } else if (MODE != kModeGateUp && warp == 2 + EW) {
+    // ------------------------------------------------------------ token-row loads (down, router)
+    // A second producer: this CTA's half of each unit's token rows (H rows,
+    // or x rows for the router), armed on the leader's stage barrier beside
+    // the weight tiles, so that the two operands' loads are issued in
+    // parallel.  The weight producer of rank 0 drains the stages at the end
+    // (a stage completes only when both producers' bytes have landed).
+    const uint64_t pol_b = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int u = pair; ok && u < num_units; u += npairs) {
+      const Unit un = get_unit<MODE>(p, u);
+      const bool sh = (MODE != kModeRouter) && un.g >= p.E;
+      const int sidx = sh ? un.g - p.E : 0;
+      const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
+      const int KB = K / kTileK;
+      const int kb0 = (MODE == kModeRouter) ? un.g * p.router_kbs : 0;
+      const int kb1 = (MODE == kModeRouter) ? min(KB, kb0 + p.router_kbs) : KB;
+      const CUtensorMap* mB = p.mapB[sh ? 1 : 0];
+      const int half = un.n >> 1;
+      const int brow0 = (sh ? sidx * p.Tp : 0) + un.row0 + static_cast<int>(rank) * half;
+      int got = 1;
+      if (lane == 0) {
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
+            got = 0;
+            break;
+          }
+          const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
+          const uint32_t fb = full_leader + 8u * stage;
+          mbar_arrive_expect_tx_cluster(fb, static_cast<uint32_t>(half) * 128u);
+          tma_load_rows<true>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, half, pol_b);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) ok = false;
+    }
   } else if (MODE == kModeGateUp && warp >= 2 + EW) {
     // ------------------------------------------------------------ row gather (this CTA's half)
     // Gather warp gw lands rows [32 gw, 32 gw + 32) of this CTA's half of
@@ -1159,6 +1269,91 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
     uint8_t* stg = epi + (warp - 2) * (kEpiBytes / EW);
+    if constexpr (MODE == kModeRouter) {
+      // Router: warp (q, half) sums experts 32 q .. + 31 of this CTA's 128
+      // (thread = expert row) over one half of the run's token columns in
+      // fp32 registers, one drained partial accumulator at a time, then
+      // writes logits[t, e] through a transpose in its staging buffer.
+      const int half = (warp - 2) >> 2;
+      uint32_t dc = 0;
+      bool ok = true;
+      for (int u = pair; ok && u < num_units; u += npairs) {
+        const Unit un = get_unit<MODE>(p, u);
+        const int KB = p.d / kTileK;
+        const int kb0 = un.g * p.router_kbs;
+        const int nkb = min(KB, kb0 + p.router_kbs) - kb0;
+        const int nd = (nkb + kRouterDrainKB - 1) / kRouterDrainKB;
+        float* const lbase = reinterpret_cast<float*>(p.out_r) + static_cast<size_t>(un.g) * p.T * p.E;
+        const int feat0 = un.wb * kWbRows + static_cast<int>(rank) * kTileRows + 32 * q;
+        const bool live = feat0 < p.E;
+        const int ncol = un.n >> 1;     // this warp's token columns [c0, c0 + ncol): a multiple of 16, <= 128
+        const int c0 = half * ncol;
+        float acc[128];
+#pragma unroll
+        for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+        for (int i = 0; i < nd; ++i) {
+          const int buf = static_cast<int>(dc % static_cast<uint32_t>(p.nbuf));
+          const uint32_t bpar = (dc / static_cast<uint32_t>(p.nbuf)) & 1u;
+          int got = 1;
+          if (lane == 0) got = mbar_wait(&tfull[buf], bpar, abort_flag, p.err, p.timeout_ns) ? 1 : 0;
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (live) {
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                static_cast<uint32_t>(buf * nmax + c0);
+            // 16 columns per round trip (the 128 sums leave room for one load)
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              if (16 * g < ncol) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(tb + static_cast<uint32_t>(16 * g), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[16 * g + j] += __uint_as_float(v[j]);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty_leader + 8u * buf);
+          ++dc;
+        }
+        if (!ok || !live) continue;
+        float* sf = reinterpret_cast<float*>(stg);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (16 * c < ncol) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sf[i * 32 + lane] = acc[16 * c + i];
+            __syncwarp();
+#pragma unroll
+            for (int rep = 0; rep < 4; ++rep) {
+              const int cc = lane + 32 * rep;
+              const int tok = cc >> 3, part = cc & 7;
+              const int t = un.row0 + c0 + 16 * c + tok;
+              const int e = feat0 + part * 4;
+              if (t < p.T) {
+                float* dst = lbase + static_cast<size_t>(t) * p.E + e;
+                const float4 vv = *reinterpret_cast<const float4*>(sf + tok * 32 + part * 4);
+                if ((p.E & 3) == 0 && e + 3 < p.E) {
+                  *reinterpret_cast<float4*>(dst) = vv;
+                } else {
+                  if (e + 0 < p.E) dst[0] = vv.x;
+                  if (e + 1 < p.E) dst[1] = vv.y;
+                  if (e + 2 < p.E) dst[2] = vv.z;
+                  if (e + 3 < p.E) dst[3] = vv.w;
+                }
+              }
+            }
+            __syncwarp();
+          }
+        }
+      }
+    } else {
     uint32_t ucount = 0;
     for (int u = pair; u < num_units; u += npairs) {
       const Unit un = get_unit<MODE>(p, u);
@@ -1315,6 +1510,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(MODE), 1)
       if (lane == 0) mbar_arrive_cluster(tempty_leader + 8u * buf);
       ++ucount;
     }
+    }
   }
 
   tc_fence_before();
@@ -1355,7 +1551,8 @@ static int launch_pair_mode(const GemmParams& prm, int grid, size_t smem, cudaSt
   static std::atomic<int> limit[64];
   const int rc = raise_smem_limit(moe_gemm_pair_kernel<MODE>, limit, static_cast<int>(smem));
   if (rc != MOE_OK) return rc;
-  return launch_chained(moe_gemm_pair_kernel<MODE>, dim3(grid), dim3(threads_of(MODE)), smem, st, prm) == cudaSuccess
+  return launch_chained(moe_gemm_pair_kernel<MODE>, dim3(grid), dim3(pair_threads_of(MODE)), smem, st, prm) ==
+                 cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
@@ -1364,6 +1561,7 @@ int launch_gemm_pair(int mode, const GemmParams& prm, int grid, size_t smem, cud
   grid &= ~1;
   if (grid < 2) return MOE_ERR_UNSUPPORTED;
   switch (mode) {
+    case kModeRouter: return launch_pair_mode<kModeRouter>(prm, grid, smem, st);
     case kModeGateUp: return launch_pair_mode<kModeGateUp>(prm, grid, smem, st);
     case kModeDown: return launch_pair_mode<kModeDown>(prm, grid, smem, st);
     default: return MOE_ERR_INVALID_ARG;

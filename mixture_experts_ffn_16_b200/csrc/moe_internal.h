@@ -88,6 +88,9 @@ struct Plan {
   int Rcap;        // routed row capacity: T*k + E*(rowpad-1), rounded to rowpad
   int nb;          // permute blocks: ceil(T / kPermBlock)
   int nmax_r;      // tokens per router work unit
+  int router_pair; // 1: the router GEMM runs on CTA pairs (256 experts x nmax_r tokens per unit)
+  int router_nwb;  // expert blocks per token run: 128 experts each (256 on CTA pairs)
+  int router_Tp;   // T rounded up to the router's row step (32 on CTA pairs: each CTA loads half a run)
   int nmax1;       // rows per gate/up work unit (MMA N max)
   int nmax2;       // rows per down work unit
   int nwbE;        // 128-row blocks of E

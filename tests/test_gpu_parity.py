@@ -63,6 +63,15 @@ MEDIUM = [
     MoEConfig("E896_like_large", T=96, d=256, E=896, k=22, f=64, S=2, fs=128, seed=21),
     MoEConfig("multi_tile_medium", T=1000, d=1024, E=64, k=8, f=256, S=1, fs=256,
               score_fn="sigmoid", bias_std=0.1, seed=22),
+    # Router GEMM on CTA pairs (256 experts per unit): E not a multiple of 256
+    # (whole 128-expert halves and parts of one past E), T not a multiple of
+    # the run (the last run partly past T); runs of 128 in two K slices, of
+    # 256 in two slices with a 224-token last run, and of 256 in one slice.
+    MoEConfig("router_pairs_128_two_slices", T=1000, d=1024, E=640, k=8, f=128, S=1, fs=128, seed=26),
+    MoEConfig("router_pairs_256_two_slices", T=2500, d=1024, E=448, k=8, f=128, S=1, fs=128,
+              score_fn="sigmoid", bias_std=0.1, seed=27),
+    MoEConfig("router_pairs_256_one_slice", T=4000, d=512, E=640, k=8, f=64, S=0, fs=0,
+              score_fn="sqrt_softplus", bias_std=0.1, seed=28),
 ]
 
 
@@ -138,6 +147,47 @@ def test_full_size_workloads(oracle_mod, parity_log, name, n_tok):
     assert rep["tokens"] == (cfg.T if n_tok is None else n_tok)
     parity_log.append(dict(case=name, check="block", **rep))
     print(name, route, rep)
+
+
+# Router logits at the largest model width (d = 7168, E = 896, the skewed
+# workload's router): the tensor cores' partial sums are drained to fp32
+# registers every 128 columns of d, so that the logit error stays small next
+# to the near-tie band of the selection rule (a relative gap of 1e-5 between
+# softmax probabilities is a gap of 1e-5 between logits).  What remains is the
+# tensor cores' accumulation within each 128-column chunk plus 56 fp32
+# additions into sums of magnitude up to about 12: measured up to 5.3e-6.  The
+# bound below is 8e-6; the selection rule itself is checked token by token
+# against the oracle (check_routing).  Single CTAs (512 tokens), CTA pairs in
+# two K slices (1536) and in one (3072).
+LOGIT_CASES = [512, 1536, 3072]
+LOGIT_ATOL = 8e-6
+
+
+@pytest.mark.parametrize("T", LOGIT_CASES)
+def test_router_logits_at_large_width(oracle_mod, T):
+    _need_gpu()
+    cfg = MoEConfig("router_logits_d7168", T=T, d=7168, E=896, k=22, f=64, S=0, fs=0,
+                    skew="zipf_rank", seed=29)
+    inp = make_inputs(cfg, device="cuda")
+    shape = api.shape_of(cfg)
+    ws = api.alloc_workspace(shape)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+    api.moe_route(shape, inp["x"], inp["W_router"], None, cfg.score_fn, cfg.norm_topk, cfg.route_scale, idx, w, ws)
+    assert api.moe_device_status(ws) == api.MOE_OK
+    _, nbytes = api.moe_workspace_region(shape, "logits")
+    split = nbytes // (T * cfg.E * 4)
+    parts = api.workspace_view(ws, shape, "logits", torch.float32, (split, T, cfg.E)).cpu()
+    gpu = parts[0].clone()
+    for s in range(1, split):
+        gpu += parts[s]                 # the slices in slice order, in fp32, as top-k sums them
+    host = oracle_args(inp)
+    o = oracle_mod.forward(host["x"], host["W_router"], k=cfg.k, score_fn=cfg.score_fn, norm_topk=cfg.norm_topk,
+                           route_scale=cfg.route_scale, route_only=True, want_logits=True)
+    err = np.abs(gpu.double().numpy() - o["logits"]).max()
+    print(f"T={T} slices={split} max|logit err|={err:.3e} max|logit|={np.abs(o['logits']).max():.3f}")
+    assert err <= LOGIT_ATOL
+    check_routing(oracle_mod, cfg, host, idx.cpu().numpy(), w.cpu().numpy())
 
 
 GATED = [

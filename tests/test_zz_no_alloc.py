@@ -60,14 +60,16 @@ def test_noalloc_route_matches_workspace_route_twice(oracle_mod, cfg):
 
 
 def test_noalloc_route_with_fewer_slices_matches_oracle(oracle_mod, parity_log):
-    """prefill_sigmoid: T * E fp32 logits (12.6 MB) fit the 16 MiB scratch, but
-    the workspace plan's two slices of d (25 MB of partial logits) do not, so
-    the call sums the logits over one slice: a different fp32 summation order
-    than moe_route, checked against the oracle by the near-tie rule."""
+    """T = 8448, d = 2048, E = 256: T * E fp32 logits (8.25 MiB) fit the 16 MiB
+    scratch, but the workspace plan's two slices of d (16.5 MiB of partial
+    logits) do not, so the call sums the logits over one slice: a different
+    fp32 summation order than moe_route, checked against the oracle by the
+    near-tie rule."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     api.load()
-    cfg = CONFIGS["prefill_sigmoid"]
+    cfg = MoEConfig("noalloc_one_slice", T=8448, d=2048, E=256, k=8, f=64, S=0, fs=0, score_fn="sigmoid",
+                    bias_std=0.1, seed=42)
     shape = api.shape_of(cfg)
     off, nbytes = api.moe_workspace_region(shape, "logits")
     assert nbytes > 16 * 2**20 >= cfg.T * cfg.E * 4         # the branch that cuts the slices
@@ -83,7 +85,7 @@ def test_noalloc_route_with_fewer_slices_matches_oracle(oracle_mod, parity_log):
                 "expert_bias": inp["expert_bias"].cpu().numpy()}
         rep = check_routing(oracle_mod, cfg, host, idx.cpu().numpy(), w.cpu().numpy())
         assert rep["tokens"] == cfg.T
-    parity_log.append(dict(case="prefill_sigmoid_noalloc", check="routing", **rep))
+    parity_log.append(dict(case="noalloc_one_slice", check="routing", **rep))
 
 
 def test_noalloc_route_refuses_shapes_beyond_its_scratch():
