@@ -978,9 +978,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      // leader: the weight producers' expect-tx arrivals of both CTAs, plus
-      // those of both CTAs' gather warps (gate/up) or token producers
-      mbar_init(full + s, MODE == kModeGateUp ? 2 + 2 * kGatherWarps : 4);
+      // leader: the weight producers' expect-tx arrivals of both CTAs (gate/
+      // up: they also count the bytes their CTA's gather warps bring), plus
+      // the token producers' (down, router)
+      mbar_init(full + s, MODE == kModeGateUp ? 2 : 4);
       mbar_init(empty + s, 1);
     }
     for (int b = 0; b < kMaxTmemBufs; ++b) {
@@ -1035,21 +1036,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
       const int kb1 = (MODE == kModeRouter) ? min(KB, kb0 + p.router_kbs) : KB;
       const CUtensorMap* mA = &p.mapA[sh ? 2 : 0];
       const int a_c2 = (MODE == kModeRouter) ? 0 : (sh ? sidx : un.g);
-      const uint32_t tx_bytes = NA * kATileBytes;
-      int got = 1;
-      if (lane == 0) {
+      // gate/up: this CTA's gathered token rows (half of the run) land on the
+      // same stage barrier without arriving on it; their bytes are expected here
+      const uint32_t tx_bytes = NA * kATileBytes + (MODE == kModeGateUp ? static_cast<uint32_t>(un.n >> 1) * 128u : 0u);
+      const int wrow = un.wb * kWbRows + static_cast<int>(rank) * kTileRows;
+      if constexpr (NA == 1) {
+        // one weight tile per stage: lane 0 alone
+        int got = 1;
+        if (lane == 0) {
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
+              got = 0;
+              break;
+            }
+            const uint32_t fb = full_leader + 8u * stage;
+            mbar_arrive_expect_tx_cluster(fb, tx_bytes);
+            tma_load_3d_pair_hint(smem_u32(smem + static_cast<size_t>(stage) * stage_bytes), mA, fb, kb * kTileK,
+                                  wrow, a_c2, pol_a);
+            ++issued;
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) ok = false;
+      } else {
+        // gate and up tile: lane 0 arms the stage, lanes 0 and 1 load one
+        // tile each (measured faster than one lane loading both)
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
-            got = 0;
+          int got = 1;
+          if (lane == 0) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns))
+              got = 0;
+            else
+              mbar_arrive_expect_tx_cluster(full_leader + 8u * stage, tx_bytes);
+          }
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
+            ok = false;
             break;
           }
-          const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
-          const uint32_t fb = full_leader + 8u * stage;
-          mbar_arrive_expect_tx_cluster(fb, tx_bytes);
-#pragma unroll
-          for (int a = 0; a < NA; ++a)
-            tma_load_3d_pair_hint(sbase + a * kATileBytes, mA + a, fb, kb * kTileK,
-                                  un.wb * kWbRows + static_cast<int>(rank) * kTileRows, a_c2, pol_a);
+          if (lane < NA)
+            tma_load_3d_pair_hint(smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + lane * kATileBytes,
+                                  mA + lane, full_leader + 8u * stage, kb * kTileK, wrow, a_c2, pol_a);
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -1057,8 +1088,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
           }
         }
       }
-      got = __shfl_sync(0xffffffffu, got, 0);
-      if (!got) ok = false;
     }
     // The leader's stage barriers count both CTAs' bytes: drain the last ones.
     if (lane == 0 && rank == 0) {
@@ -1218,8 +1247,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
     // ------------------------------------------------------------ row gather (this CTA's half)
     // Gather warp gw lands rows [32 gw, 32 gw + 32) of this CTA's half of
     // the token tile with 4-row tensor gathers (one 128-byte row piece each,
-    // swizzled by the map like a tiled load); its lane 0 arms the leader's
-    // stage barrier with their bytes and issues them.
+    // swizzled by the map like a tiled load), one per lane, counted on the
+    // leader's stage barrier; this CTA's weight producer expects their bytes
+    // (a gather may land before that arrival: the barrier's transaction
+    // count then runs below zero until it, and the phase cannot complete
+    // while the arrival is pending).
     const int gw = warp - (2 + EW);
     const uint64_t pol_x = policy_evict_last();
     int stage = 0;
@@ -1233,31 +1265,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
       const int rb = un.row0 + static_cast<int>(rank) * half + 32 * gw;
       // clamped: a row never reads outside x, even for an invalid routing
       const int my = (lane < nr) ? min(max(sh ? rb + lane : __ldg(p.perm + rb + lane), 0), p.T - 1) : 0;
-      int tk[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) tk[j] = __shfl_sync(0xffffffffu, my, j);
+      // lane j < nr / 4 gathers rows 4 j .. 4 j + 3 of the warp's 32
+      const int t0 = __shfl_sync(0xffffffffu, my, (4 * lane) & 31);
+      const int t1 = __shfl_sync(0xffffffffu, my, (4 * lane + 1) & 31);
+      const int t2 = __shfl_sync(0xffffffffu, my, (4 * lane + 2) & 31);
+      const int t3 = __shfl_sync(0xffffffffu, my, (4 * lane + 3) & 31);
       const int KB = p.d / kTileK;
       for (int kb = 0; kb < KB; ++kb) {
         int got = 1;
-        if (lane == 0) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) {
-            got = 0;
-          } else {
-            const uint32_t fb = full_leader + 8u * stage;
-            mbar_arrive_expect_tx_cluster(fb, static_cast<uint32_t>(nr) * 128u);
-            const uint32_t dst = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + NA * kATileBytes +
-                                 static_cast<uint32_t>(32 * gw) * 128u;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (4 * j < nr)
-                tma_gather4_pair(dst + static_cast<uint32_t>(4 * j) * 128u, &p.mapX, fb, kb * kTileK, tk[4 * j],
-                                 tk[4 * j + 1], tk[4 * j + 2], tk[4 * j + 3], pol_x);
-          }
-        }
+        // the stage is free once its previous MMAs are done; the weight
+        // producer's arrival expects these bytes (before or after they land)
+        if (lane == 0 && !mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, p.timeout_ns)) got = 0;
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) {
           ok = false;
           break;
+        }
+        // its gathers are issued by several lanes at once
+        if (4 * lane < nr) {
+          const uint32_t dst = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + NA * kATileBytes +
+                               static_cast<uint32_t>(32 * gw + 4 * lane) * 128u;
+          tma_gather4_pair(dst, &p.mapX, full_leader + 8u * stage, kb * kTileK, t0, t1, t2, t3, pol_x);
         }
         if (++stage == S) {
           stage = 0;

@@ -5,7 +5,9 @@
 // slice order), forms the scores and selection keys in registers, and picks the k
 // largest keys by k rounds of a warp-wide arg-max (ties go to the lower expert
 // index, matching a stable descending sort); each round reduces the lanes'
-// best keys with two warp reductions.
+// best keys with two warp reductions.  A lane keeps its keys in groups of up
+// to 8 with each group's best, so after a round only the winning lane
+// rescans one group (instead of every lane rescanning all of its keys).
 //
 //   softmax       : key = logit (same order as the softmax probability);
 //                   w_j = exp(l_j - l_max) / (norm ? sum over picks : sum over all E)
@@ -43,6 +45,25 @@ __device__ __forceinline__ uint32_t key_code(float key) {
   if (key != key) return kKeyFloor;            // NaN
   const uint32_t ub = __float_as_uint(key + 0.0f);
   return (ub & 0x80000000u) ? ~ub : (ub | 0x80000000u);
+}
+
+// Group g (slots g*GS .. g*GS + GS - 1) of a lane's codes: drop slot ws (if
+// it is in the group) and recompute the group's best code and slot.
+template <int NPL, int GS, int g>
+__device__ __forceinline__ void rescan_group(uint32_t (&code)[NPL], uint32_t (&gc)[NPL / GS], int (&gs)[NPL / GS],
+                                             int ws) {
+  if constexpr (g < NPL / GS) {
+    gc[g] = 0u;
+    gs[g] = 0;
+#pragma unroll
+    for (int jj = 0; jj < GS; ++jj) {
+      if (g * GS + jj == ws) code[g * GS + jj] = 0u;
+      if (code[g * GS + jj] > gc[g]) {
+        gc[g] = code[g * GS + jj];
+        gs[g] = g * GS + jj;
+      }
+    }
+  }
 }
 
 template <int NPL>   // keys per lane: E <= 32 * NPL
@@ -113,28 +134,68 @@ topk_kernel(const float* __restrict__ logits, int nsplit, const float* __restric
     }
   }
 
-  int my_idx = 0;    // lane j keeps the j-th pick
-  for (int j = 0; j < k; ++j) {
-    // this lane's best remaining key (the lower expert index on equal codes)
-    uint32_t bc = 0u;
-    int bi = 0x7fffffff;
+  // Groups of GS consecutive slots (slot i = expert lane + 32 i), each with
+  // its best code and slot (the lower slot, i.e. the lower expert, on equal
+  // codes); the lane's best is the best of its groups in slot order.
+  constexpr int GS = NPL < 8 ? NPL : 8;
+  constexpr int G = NPL / GS;
+  static_assert(G <= 8, "at most 8 groups");
+  uint32_t gc[G];
+  int gs[G];
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      if (code[i] > bc) {
-        bc = code[i];
-        bi = lane + 32 * i;
+  for (int g = 0; g < G; ++g) {
+    gc[g] = 0u;
+    gs[g] = 0;
+#pragma unroll
+    for (int jj = 0; jj < GS; ++jj) {
+      if (code[g * GS + jj] > gc[g]) {
+        gc[g] = code[g * GS + jj];
+        gs[g] = g * GS + jj;
       }
     }
+  }
+  uint32_t bc = 0u;   // this lane's best remaining code (0: none left)
+  int bs = 0;         // ... and its slot
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    if (gc[g] > bc) {
+      bc = gc[g];
+      bs = gs[g];
+    }
+  }
+
+  int my_idx = 0;    // lane j keeps the j-th pick
+  for (int j = 0; j < k; ++j) {
     // Warp arg-max in two reductions: the largest code, then the lowest
     // expert index among the lanes that hold it.  k <= E leaves at least one
     // unpicked expert, whose code is >= kKeyFloor > 0, so the winner is one.
     const uint32_t cmax = __reduce_max_sync(0xffffffffu, bc);
-    bi = static_cast<int>(__reduce_min_sync(0xffffffffu, bc == cmax ? static_cast<uint32_t>(bi) : 0x7fffffffu));
-    // Remove the winner (its owner lane), record it in lane j.
-#pragma unroll
-    for (int i = 0; i < NPL; ++i)
-      if (lane + 32 * i == bi) code[i] = 0u;
+    const int bi = static_cast<int>(
+        __reduce_min_sync(0xffffffffu, bc == cmax ? static_cast<uint32_t>(lane + 32 * bs) : 0x7fffffffu));
     if (lane == j) my_idx = bi;
+    // The owner lane removes the winner and rescans the winner's group.
+    if ((bi & 31) == lane) {
+      const int ws = bi >> 5;
+      switch (ws / GS) {   // G <= 8; a switch keeps every index static
+        case 0: rescan_group<NPL, GS, 0>(code, gc, gs, ws); break;
+        case 1: rescan_group<NPL, GS, 1>(code, gc, gs, ws); break;
+        case 2: rescan_group<NPL, GS, 2>(code, gc, gs, ws); break;
+        case 3: rescan_group<NPL, GS, 3>(code, gc, gs, ws); break;
+        case 4: rescan_group<NPL, GS, 4>(code, gc, gs, ws); break;
+        case 5: rescan_group<NPL, GS, 5>(code, gc, gs, ws); break;
+        case 6: rescan_group<NPL, GS, 6>(code, gc, gs, ws); break;
+        default: rescan_group<NPL, GS, 7>(code, gc, gs, ws); break;
+      }
+      bc = 0u;
+      bs = 0;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        if (gc[g] > bc) {
+          bc = gc[g];
+          bs = gs[g];
+        }
+      }
+    }
   }
 
   float s = 0.0f;
