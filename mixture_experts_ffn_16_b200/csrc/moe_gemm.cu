@@ -978,10 +978,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      // leader: the weight producers' expect-tx arrivals of both CTAs (gate/
-      // up: they also count the bytes their CTA's gather warps bring), plus
-      // the token producers' (down, router)
-      mbar_init(full + s, MODE == kModeGateUp ? 2 : 4);
+      // leader: the weight producers' expect-tx arrivals of both CTAs; each
+      // also counts the bytes its CTA's token rows bring (gathered by the
+      // gather warps, or loaded by the token producer)
+      mbar_init(full + s, 2);
       mbar_init(empty + s, 1);
     }
     for (int b = 0; b < kMaxTmemBufs; ++b) {
@@ -1036,9 +1036,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
       const int kb1 = (MODE == kModeRouter) ? min(KB, kb0 + p.router_kbs) : KB;
       const CUtensorMap* mA = &p.mapA[sh ? 2 : 0];
       const int a_c2 = (MODE == kModeRouter) ? 0 : (sh ? sidx : un.g);
-      // gate/up: this CTA's gathered token rows (half of the run) land on the
-      // same stage barrier without arriving on it; their bytes are expected here
-      const uint32_t tx_bytes = NA * kATileBytes + (MODE == kModeGateUp ? static_cast<uint32_t>(un.n >> 1) * 128u : 0u);
+      // this CTA's token rows (half of the run) land on the same stage barrier
+      // without arriving on it; their bytes are expected here
+      const uint32_t tx_bytes = NA * kATileBytes + static_cast<uint32_t>(un.n >> 1) * 128u;
       const int wrow = un.wb * kWbRows + static_cast<int>(rank) * kTileRows;
       if constexpr (NA == 1) {
         // one weight tile per stage: lane 0 alone
@@ -1204,10 +1204,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
   } else if (MODE != kModeGateUp && warp == 2 + EW) {
     // ------------------------------------------------------------ token-row loads (down, router)
     // A second producer: this CTA's half of each unit's token rows (H rows,
-    // or x rows for the router), armed on the leader's stage barrier beside
+    // or x rows for the router), counted on the leader's stage barrier beside
     // the weight tiles, so that the two operands' loads are issued in
-    // parallel.  The weight producer of rank 0 drains the stages at the end
-    // (a stage completes only when both producers' bytes have landed).
+    // parallel.  It does not arrive: the weight producer's arrival expects
+    // these bytes too (they may land first; the transaction count then runs
+    // below zero until it).  The weight producer of rank 0 drains the stages
+    // at the end (a stage completes only when all of its bytes have landed).
     const uint64_t pol_b = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
@@ -1231,9 +1233,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
             break;
           }
           const uint32_t sbase = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes);
-          const uint32_t fb = full_leader + 8u * stage;
-          mbar_arrive_expect_tx_cluster(fb, static_cast<uint32_t>(half) * 128u);
-          tma_load_rows<true>(sbase + NA * kATileBytes, mB, fb, kb * kTileK, brow0, half, pol_b);
+          tma_load_rows<true>(sbase + NA * kATileBytes, mB, full_leader + 8u * stage, kb * kTileK, brow0, half,
+                              pol_b);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
