@@ -468,11 +468,23 @@ def time_e2e(run, K, W, world):
         if st_chk != api.MOE_OK:
             raise RuntimeError(f"device status after e2e: {api.status_string(st_chk)}")
     e2e_ms = max_over_ranks(max(e0.elapsed_time(ev) for ev in ends), world)
+    # Latency of one call on its own (nothing else in flight): copies in,
+    # the block, copies out, on one stream; median of a few calls.
+    lat = []
+    for i in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(lanes[0]["stream"])
+        host_step(0)
+        b.record(lanes[0]["stream"])
+        torch.cuda.synchronize()
+        lat.append(a.elapsed_time(b))
+    lat_ms = max_over_ranks(statistics.median(lat), world)
     del lanes
     return {"value": world * cfg.T * K / (e2e_ms / 1e3), "unit": "tokens/s",
             "h2d_bytes_per_step": cfg.T * cfg.d * 2,
             "d2h_bytes_per_step": cfg.T * cfg.d * 2 + cfg.T * cfg.k * 8,
-            "streams": NL, "ms_per_step": e2e_ms / K}
+            "streams": NL, "ms_per_step": e2e_ms / K, "latency_ms_per_call": lat_ms}
 
 
 def extra_workloads(args, main_name, dev, world, rank):
