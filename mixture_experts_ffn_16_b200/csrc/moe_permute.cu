@@ -7,9 +7,9 @@
 //             block's offset inside the expert's segment) and the expert's
 //             count; then an exclusive scan over experts of the padded segment
 //             sizes (rows stay in expert order), a rank of every expert by
-//             padded rows (largest first), exclusive scans in rank order of
-//             the GEMM work-unit counts; writes the work lists (largest
-//             expert first) and fills the padding rows.
+//             padded rows, exclusive scans of the GEMM work-unit counts in
+//             list order (largest, smallest, 2nd largest, ...); writes the
+//             work lists and fills the padding rows.
 //   scatter : recomputes the masks (each of the ceil(k/2) CTAs of a block
 //             places two slots of its tokens); a (token, slot) pair's row is
 //             segment start + block offset + popcount of the lower lanes of
@@ -134,7 +134,7 @@ struct ScanArgs {
 
 __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) {
   // Padded rows of every expert, then (by rank) its unit counts and their
-  // exclusive offsets: the work lists run largest expert first.
+  // exclusive offsets, in the work lists' interleaved size order.
   __shared__ __align__(16) int s_key[kMaxE];
   __shared__ int s_u1[kMaxE], s_u2[kMaxE];
   chain_wait();
@@ -173,10 +173,13 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) 
   int3 tot;
   const int3 ex = block_exclusive_scan3(make_int3(sp, 0, 0), &tot);
   const int tot_rows = tot.x;
-  // Rank of each expert in the work lists: more padded rows first, then the
-  // lower expert index (a strict order, so ranks are 0..E-1).  Each work
-  // list then starts with the biggest experts, so the units of the last
-  // rounds over the SMs are the smallest.  Rows keep the expert order.
+  // Position of each expert in the work lists: experts ranked by padded rows
+  // (more first, then the lower expert index: a strict order, ranks 0..E-1),
+  // then interleaved from both ends of that ranking - largest, smallest, 2nd
+  // largest, 2nd smallest, ...  Large experts' units keep the tensor cores
+  // busy while small experts' units, which stream their weights once for few
+  // tokens, run beside them instead of all together at the end.  Rows keep
+  // the expert order.
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = (i < per) ? threadIdx.x * per + i : a.E;
@@ -191,6 +194,8 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(ScanArgs a) 
              (k4.z > key || (k4.z == key && e2 + 2 < e)) + (k4.w > key || (k4.w == key && e2 + 3 < e));
       }
       for (int e2 = E4; e2 < a.E; ++e2) r += (s_key[e2] > key || (s_key[e2] == key && e2 < e));
+      // list position: largest, smallest, 2nd largest, 2nd smallest, ...
+      r = (r < (a.E + 1) / 2) ? 2 * r : 2 * (a.E - 1 - r) + 1;
       rank[i] = r;
       s_u1[r] = u1[i];
       s_u2[r] = u2[i];
