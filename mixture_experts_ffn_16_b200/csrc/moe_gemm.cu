@@ -120,6 +120,14 @@ __device__ __forceinline__ Unit get_unit(const GemmParams& p, int u) {
   return un;
 }
 
+// The it-th work unit of CTA (or CTA pair) p of P: round it covers units
+// it*P .. it*P + P - 1, handed out in forward order on even rounds and in
+// backward order on odd ones, so that a CTA that got one of the larger
+// units of a round (the lists run from large to small units, interleaved)
+// gets one of the smaller ones in the next.  Increasing in it for every p,
+// so a loop may stop at the first index past the list.
+__device__ __forceinline__ int snake_unit(int it, int p, int P) { return it * P + ((it & 1) ? P - 1 - p : p); }
+
 // Bounded wait that ignores the abort flag: used only to drain work this block
 // itself put in flight before it leaves.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
@@ -349,7 +357,8 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
     uint32_t phase = 0;
     uint32_t issued = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+    for (int it = 0, u = snake_unit(0, blockIdx.x, gridDim.x); ok && u < num_units;
+         u = snake_unit(++it, blockIdx.x, gridDim.x)) {
       const Unit un = get_unit<MODE>(p, u);
       const bool sh = (MODE != kModeRouter) && un.g >= p.E;
       const int sidx = sh ? un.g - p.E : 0;
@@ -432,7 +441,8 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
         // into fp32 registers by the epilogue, so no tensor-core accumulation
         // chain is longer than 4 * kRouterDrainKB MMA steps.
         uint32_t dc = 0;
-        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        for (int it = 0, u = snake_unit(0, blockIdx.x, gridDim.x); ok && u < num_units;
+             u = snake_unit(++it, blockIdx.x, gridDim.x)) {
           const Unit un = get_unit<MODE>(p, u);
           const int KB = p.d / kTileK;
           const int kb0 = un.g * p.router_kbs;
@@ -475,7 +485,8 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
           }
         }
       } else {
-        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        for (int it = 0, u = snake_unit(0, blockIdx.x, gridDim.x); ok && u < num_units;
+             u = snake_unit(++it, blockIdx.x, gridDim.x)) {
           const Unit un = get_unit<MODE>(p, u);
           const bool sh = (MODE != kModeRouter) && un.g >= p.E;
           const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
@@ -561,7 +572,8 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
     uint32_t rph = 0, mph = 0;
     int pms = -1;                    // MMA stage written but not yet published
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+    for (int it = 0, u = snake_unit(0, blockIdx.x, gridDim.x); ok && u < num_units;
+         u = snake_unit(++it, blockIdx.x, gridDim.x)) {
       const Unit un = get_unit<MODE>(p, u);
       const bool sh = un.g >= p.E;
       const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
@@ -632,7 +644,8 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
       int ts = 0;
       uint32_t tph = 0, issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      for (int it = 0, u = snake_unit(0, blockIdx.x, gridDim.x); ok && u < num_units;
+           u = snake_unit(++it, blockIdx.x, gridDim.x)) {
         const Unit un = get_unit<MODE>(p, u);
         const bool sh = un.g >= p.E;
         const int sidx = sh ? un.g - p.E : 0;
@@ -679,7 +692,8 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+    for (int it = 0, u = snake_unit(0, blockIdx.x, gridDim.x); ok && u < num_units;
+         u = snake_unit(++it, blockIdx.x, gridDim.x)) {
       const Unit un = get_unit<MODE>(p, u);
       const bool sh = un.g >= p.E;
       const int nr = un.n >> 4;                    // rows of this thread
@@ -727,7 +741,8 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
       // logits[t, e] (thread = expert row, column = token).
       uint32_t dc = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      for (int it = 0, u = snake_unit(0, blockIdx.x, gridDim.x); ok && u < num_units;
+           u = snake_unit(++it, blockIdx.x, gridDim.x)) {
         const Unit un = get_unit<MODE>(p, u);
         const int KB = p.d / kTileK;
         const int kb0 = un.g * p.router_kbs;
@@ -809,7 +824,8 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
     } else {
       uint32_t ucount = 0;
       uint32_t ech = 0;                 // chunks stored by this warp (staging slot = ech & 1)
-      for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      for (int it = 0, u = snake_unit(0, blockIdx.x, gridDim.x); u < num_units;
+           u = snake_unit(++it, blockIdx.x, gridDim.x)) {
         const Unit un = get_unit<MODE>(p, u);
         const bool sh = (MODE != kModeRouter) && un.g >= p.E;
         const int sidx = sh ? un.g - p.E : 0;
@@ -1025,7 +1041,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
     uint32_t phase = 0;
     uint32_t issued = 0;
     bool ok = true;
-    for (int u = pair; ok && u < num_units; u += npairs) {
+    for (int it = 0, u = snake_unit(0, pair, npairs); ok && u < num_units; u = snake_unit(++it, pair, npairs)) {
       const Unit un = get_unit<MODE>(p, u);
       const bool sh = (MODE != kModeRouter) && un.g >= p.E;
       const int sidx = sh ? un.g - p.E : 0;
@@ -1111,7 +1127,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
         // registers by both CTAs' epilogues (as in the single-CTA router),
         // through nbuf buffers of nmax columns.
         uint32_t dc = 0;
-        for (int u = pair; ok && u < num_units; u += npairs) {
+        for (int it = 0, u = snake_unit(0, pair, npairs); ok && u < num_units; u = snake_unit(++it, pair, npairs)) {
           const Unit un = get_unit<MODE>(p, u);
           const int KB = p.d / kTileK;
           const int kb0 = un.g * p.router_kbs;
@@ -1155,7 +1171,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
           }
         }
       }
-      for (int u = pair; MODE != kModeRouter && ok && u < num_units; u += npairs) {
+      for (int it = 0, u = snake_unit(0, pair, npairs); MODE != kModeRouter && ok && u < num_units;
+           u = snake_unit(++it, pair, npairs)) {
         const Unit un = get_unit<MODE>(p, u);
         const bool sh = un.g >= p.E;
         const int K = (MODE == kModeDown) ? (sh ? p.fs : p.f) : p.d;
@@ -1214,7 +1231,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int u = pair; ok && u < num_units; u += npairs) {
+    for (int it = 0, u = snake_unit(0, pair, npairs); ok && u < num_units; u = snake_unit(++it, pair, npairs)) {
       const Unit un = get_unit<MODE>(p, u);
       const bool sh = (MODE != kModeRouter) && un.g >= p.E;
       const int sidx = sh ? un.g - p.E : 0;
@@ -1258,7 +1275,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int u = pair; ok && u < num_units; u += npairs) {
+    for (int it = 0, u = snake_unit(0, pair, npairs); ok && u < num_units; u = snake_unit(++it, pair, npairs)) {
       const Unit un = get_unit<MODE>(p, u);
       const bool sh = un.g >= p.E;
       const int half = un.n >> 1;
@@ -1306,7 +1323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
       const int half = (warp - 2) >> 2;
       uint32_t dc = 0;
       bool ok = true;
-      for (int u = pair; ok && u < num_units; u += npairs) {
+      for (int it = 0, u = snake_unit(0, pair, npairs); ok && u < num_units; u = snake_unit(++it, pair, npairs)) {
         const Unit un = get_unit<MODE>(p, u);
         const int KB = p.d / kTileK;
         const int kb0 = un.g * p.router_kbs;
@@ -1384,7 +1401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
       }
     } else {
     uint32_t ucount = 0;
-    for (int u = pair; u < num_units; u += npairs) {
+    for (int it = 0, u = snake_unit(0, pair, npairs); u < num_units; u = snake_unit(++it, pair, npairs)) {
       const Unit un = get_unit<MODE>(p, u);
       const bool sh = un.g >= p.E;
       const int sidx = sh ? un.g - p.E : 0;
