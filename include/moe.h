@@ -300,8 +300,9 @@ MOE_API int moe_experts_forward(const moe_shape *shape, const void *x, const int
  *                                load fewer bytes per SM; P <= 16)
  *   MOE_WS_COUNTS   int32 [E]    tokens per expert (after moe_permute)
  *   MOE_WS_OFFSETS  int32 [E+1]  first row of each expert's segment; segments
- *                                are padded to p rows (p = 16, or 32 when
- *                                experts average 256+ rows); [E] = total rows
+ *                                are padded to p rows (p = 16, or 32 when the
+ *                                expert GEMMs run on CTA pairs: experts of 96+
+ *                                rows on average); [E] = total rows
  *   MOE_WS_PERM     int32 [rows] token of each routed row (padding rows: 0)
  *   MOE_WS_ROW_W    fp32 [rows]  combine weight of each routed row (padding: 0)
  *   MOE_WS_INV      int32 [T,k]  row of each (token, slot)
@@ -312,6 +313,16 @@ MOE_API int moe_experts_forward(const moe_shape *shape, const void *x, const int
  *   MOE_WS_X_STAGE  bf16 [T,d]      token rows the library staged: x copied
  *                                   from the host (moe_forward_host) or the
  *                                   normalised x (moe_forward_prenorm)
+ *   MOE_WS_WORK_COUNTS  int32 [4]   after moe_permute: gate/up work units U1,
+ *                                   down work units U2, routed rows, a tag of
+ *                                   the plan that wrote the lists
+ *   MOE_WS_WORK_GATE_UP int32 [U1,4] gate/up work units {group, weight block,
+ *                                   first row, rows}: groups >= E are the
+ *                                   shared experts (first in the list), whose
+ *                                   rows index [0, Tp); routed units follow
+ *                                   expert by expert, largest, smallest, 2nd
+ *                                   largest, 2nd smallest, ... by padded rows
+ *   MOE_WS_WORK_DOWN    int32 [U2,4] the same for the down GEMM
  * Writes the region's byte offset in the workspace and its capacity in bytes.
  * Returns MOE_OK, or MOE_ERR_INVALID_ARG for a bad shape, region or pointer. */
 #define MOE_WS_LOGITS   0
@@ -325,6 +336,9 @@ MOE_API int moe_experts_forward(const moe_shape *shape, const void *x, const int
 #define MOE_WS_Y        8
 #define MOE_WS_Y_SHARED 9
 #define MOE_WS_X_STAGE  10
+#define MOE_WS_WORK_COUNTS  11
+#define MOE_WS_WORK_GATE_UP 12
+#define MOE_WS_WORK_DOWN    13
 MOE_API int moe_workspace_region(const moe_shape *shape, int region, size_t *offset, size_t *bytes);
 
 /* Synchronises `stream`, then returns MOE_ERR_DEVICE_TIMEOUT if a kernel of a

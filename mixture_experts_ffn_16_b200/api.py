@@ -28,7 +28,8 @@ MOE_ERR_NONFINITE = -7
 SCORE_FNS = {"softmax": 0, "sigmoid": 1, "sqrt_softplus": 2}
 
 WS_REGIONS = {"logits": 0, "counts": 1, "offsets": 2, "perm": 3, "row_w": 4, "inv": 5,
-              "h": 6, "h_shared": 7, "y": 8, "y_shared": 9, "x_stage": 10}
+              "h": 6, "h_shared": 7, "y": 8, "y_shared": 9, "x_stage": 10,
+              "work_counts": 11, "work_gate_up": 12, "work_down": 13}
 
 EXPORTED = ["moe_version", "moe_status_string", "moe_workspace_bytes", "moe_forward",
             "moe_forward_host", "moe_route", "moe_permute", "moe_expert_gate_up", "moe_expert_down",

@@ -891,6 +891,9 @@ int moe_workspace_region(const moe_shape* shape, int region, size_t* offset, siz
     case MOE_WS_Y: *offset = p.Yr; *bytes = R * p.d * 2; break;
     case MOE_WS_Y_SHARED: *offset = p.Ys; *bytes = S * Tp * p.d * 2; break;
     case MOE_WS_X_STAGE: *offset = p.xstage; *bytes = T * p.d * 2; break;
+    case MOE_WS_WORK_COUNTS: *offset = p.nunits; *bytes = 16; break;
+    case MOE_WS_WORK_GATE_UP: *offset = p.units1; *bytes = static_cast<size_t>(p.U1cap) * 16; break;
+    case MOE_WS_WORK_DOWN: *offset = p.units2; *bytes = static_cast<size_t>(p.U2cap) * 16; break;
     default: return MOE_ERR_INVALID_ARG;
   }
   return MOE_OK;

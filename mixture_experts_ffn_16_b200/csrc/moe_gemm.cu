@@ -956,7 +956,11 @@ __global__ void __launch_bounds__(threads_of(MODE, F8), 1) moe_gemm_kernel(const
 // The leader CTA (rank 0) issues the MMAs; loads of both CTAs complete on the
 // leader's stage barrier (cta_group::2 tensor loads and, gate/up, 4-row
 // tensor gathers of the token rows; no multicast); the leader's commits
-// arrive on the barrier at the same offset in both CTAs.  The gathers move a
+// arrive on the barrier at the same offset in both CTAs.  A stage completes
+// on two arrivals, those of the two CTAs' weight producers, each expecting
+// its CTA's weight and token bytes; the token rows come from the gather
+// warps (gate/up) or a second producer warp (down, router), which do not
+// arrive.  Work units are handed to the pairs in snake order (snake_unit).  The gathers move a
 // 128-byte row piece per row where cp.async moves 16 bytes per request: with
 // 16-byte requests the gather's request rate bounded the pair gate/up
 // (measured: 7.2 -> 6.3 ms at T = 16384, d = 7168, E = 896, k = 22).  A

@@ -232,6 +232,36 @@ def test_router_logit_slices(lib, name):
     assert 1 <= slices <= min(16, c.d // 64)
 
 
+# The router tiling each workload gets (K slices of d): small batches split d
+# to fill the SMs (tiny, decode); prefill_softmax reads fewer W_router bytes
+# per SM with two slices of single-CTA units; prefill_sigmoid and
+# large_imbalanced run on CTA pairs of 256 experts x 256 tokens, the latter in
+# two slices to spread its 256 pair-units over the pairs evenly.
+ROUTER_SLICES = {"tiny": 4, "prefill_softmax": 2, "prefill_sigmoid": 1, "decode_sqrt_softplus": 8,
+                 "large_imbalanced": 2}
+
+
+@pytest.mark.parametrize("name", list(ROUTER_SLICES))
+def test_router_plan_of_each_workload(lib, name):
+    c = CONFIGS[name]
+    _, nb = api.moe_workspace_region(api.shape_of(c), "logits")
+    assert nb // (c.T * c.E * 4) == ROUTER_SLICES[name]
+
+
+def test_work_list_regions_hold_the_largest_lists():
+    """The work-list regions hold the most units any routing can produce:
+    every routed row in its own run plus one partial run per expert, per
+    weight block, plus the shared experts' runs."""
+    c = CONFIGS["large_imbalanced"]
+    s = api.shape_of(c)
+    assert api.moe_workspace_region(s, "work_counts")[1] == 16
+    rows_cap = c.T * c.k + c.E * 31
+    for name, nwb, nwbs in (("work_gate_up", c.f // 128, c.fs // 128), ("work_down", c.d // 256, c.d // 256)):
+        _, nb = api.moe_workspace_region(s, name)
+        assert nb % 16 == 0
+        assert nb // 16 >= nwb * (rows_cap // 128) + c.S * nwbs * (c.T // 128)
+
+
 def test_binding_marshalling_checks():
     """The Python binding checks device, dtype, shape and layout before it
     hands a pointer to the library."""

@@ -121,6 +121,93 @@ def test_permute_matches_brute_force_counting_sort(T, E, k):
             assert exp_roff[idx_n[t, j]] <= r < exp_roff[idx_n[t, j]] + exp_counts[idx_n[t, j]]
 
 
+def _skewed_routing(T, E, k, seed):
+    """k distinct experts per token, drawn with probability proportional to
+    rank^-1.1 over a shuffled ranking, so that expert sizes vary by an order
+    of magnitude and some experts get no token."""
+    rng = np.random.default_rng(seed)
+    p = 1.0 / (1.0 + rng.permutation(E)) ** 1.1
+    p /= p.sum()
+    idx = np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+    w = rng.random((T, k), dtype=np.float32)
+    return torch.from_numpy(idx), torch.from_numpy(w)
+
+
+def _check_work_list(units, E, seg, label):
+    """units: int [U, 4] {group, weight block, first row, rows}; seg(g) = the
+    group's row range.  Every group's runs tile its range once for each weight
+    block, the shared groups (>= E) come first, each routed group's units are
+    contiguous; returns the routed groups in list order."""
+    groups = units[:, 0]
+    shared = groups >= E
+    if shared.any():
+        assert shared[:shared.sum()].all(), label + ": shared units first"
+    order, seen = [], set()
+    prev = None
+    for g in groups[~shared]:
+        g = int(g)
+        if g != prev:
+            assert g not in seen, f"{label}: expert {g}'s units are not contiguous"
+            seen.add(g)
+            order.append(g)
+            prev = g
+    nwb = None
+    for g in np.unique(groups):
+        sel = units[groups == g]
+        lo, hi = seg(int(g))
+        wbs = np.unique(sel[:, 1])
+        assert np.array_equal(wbs, np.arange(len(wbs))), f"{label}: group {g} weight blocks {wbs}"
+        if g < E:
+            nwb = len(wbs) if nwb is None else nwb
+            assert len(wbs) == nwb, f"{label}: routed groups with different weight-block counts"
+        for wb in wbs:
+            runs = sel[sel[:, 1] == wb]
+            runs = runs[np.argsort(runs[:, 2])]
+            assert runs[0, 2] == lo and (runs[:-1, 2] + runs[:-1, 3] == runs[1:, 2]).all() \
+                and runs[-1, 2] + runs[-1, 3] == hi, f"{label}: group {g} block {wb} runs {runs.tolist()} vs [{lo}, {hi})"
+            assert (runs[:, 3] > 0).all() and (runs[:, 3] % 16 == 0).all()
+    return order
+
+
+@pytest.mark.parametrize("T,E,k,S", [(3000, 40, 4, 2), (500, 64, 2, 1), (200, 300, 6, 0)])
+def test_work_lists_tile_every_segment_in_interleaved_size_order(T, E, k, S):
+    """After moe_permute, the gate/up and down work lists cover each expert's
+    padded row segment once per weight block with runs of at most 256 rows,
+    the shared experts' rows [0, Tp) likewise and first, and the
+    routed experts in the order largest, smallest, 2nd largest, 2nd smallest,
+    ... by padded rows (ties: lower expert index first), each expert's units
+    together.  Cases: CTA pairs (300 rows per expert), single CTAs, and many
+    empty experts."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    shape = api.make_shape(T, 256, E, k, 384, S, 256 if S else 0)
+    ws = api.alloc_workspace(shape)
+    ws.zero_()
+    idx, w = _skewed_routing(T, E, k, seed=T + E)
+    api.moe_permute(shape, idx.cuda(), w.cuda(), ws)
+    torch.cuda.synchronize()
+    assert api.moe_device_status(ws) == api.MOE_OK
+    nun = api.workspace_view(ws, shape, "work_counts", torch.int32, (4,)).cpu().numpy()
+    roff = api.workspace_view(ws, shape, "offsets", torch.int32, (E + 1,)).cpu().numpy().astype(np.int64)
+    pad = roff[1:] - roff[:-1]
+    assert nun[2] == roff[E]
+    for name, n in (("work_gate_up", nun[0]), ("work_down", nun[1])):
+        units = api.workspace_view(ws, shape, name, torch.int32, (int(n), 4)).cpu().numpy().astype(np.int64)
+        assert units[:, 3].max() <= 256
+        sh = units[units[:, 0] >= E]
+        assert set(np.unique(sh[:, 0]).tolist()) == set(range(E, E + S))
+        tp = int((sh[:, 2] + sh[:, 3]).max()) if S else 0          # T rounded up to the row padding
+        assert S == 0 or tp in (-(-T // 16) * 16, -(-T // 32) * 32)
+        seg = lambda g: (0, tp) if g >= E else (int(roff[g]), int(roff[g + 1]))
+        order = _check_work_list(units, E, seg, name)
+        rank = sorted(range(E), key=lambda e: (-pad[e], e))
+        pos = [2 * r if r < (E + 1) // 2 else 2 * (E - 1 - r) + 1 for r in range(E)]
+        expect = [None] * E
+        for r, e in enumerate(rank):
+            expect[pos[r]] = e
+        assert order == [e for e in expect if pad[e] > 0], name
+
+
 def test_invalid_routing_is_reported_not_faulted():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
