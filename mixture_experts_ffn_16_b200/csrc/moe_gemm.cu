@@ -1303,8 +1303,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads_of(MODE
           ok = false;
           break;
         }
-        // its gathers are issued by several lanes at once
-        if (4 * lane < nr) {
+        if (sh) {
+          // a shared expert reads its token rows in order: one tiled load of
+          // this CTA's half of the run (rows past T read as zeros; their
+          // outputs are never combined)
+          if (gw == 0 && lane == 0)
+            tma_load_rows<true>(smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + NA * kATileBytes,
+                                p.mapB[0], full_leader + 8u * stage, kb * kTileK,
+                                un.row0 + static_cast<int>(rank) * half, half, pol_x);
+        } else if (4 * lane < nr) {
+          // the gathers are issued by several lanes at once
           const uint32_t dst = smem_u32(smem + static_cast<size_t>(stage) * stage_bytes) + NA * kATileBytes +
                                static_cast<uint32_t>(32 * gw + 4 * lane) * 128u;
           tma_gather4_pair(dst, &p.mapX, full_leader + 8u * stage, kb * kTileK, t0, t1, t2, t3, pol_x);
